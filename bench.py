@@ -1,0 +1,420 @@
+"""Benchmark of the MACaQ W4A4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward pass of the layer's hot path over one batch: the online per-channel
+scale + FWHT-32 + MXFP4 quantisation of the bf16 activations feeding the block-scaled
+MXFP4 GEMM (macaq_w4a4_linear), on the Llama-3-8B-shaped MLP up projection at prefill
+(M=2048, K=4096, N=14336) with seeded synthetic inputs (workloads.py).  The weight fold is
+offline and timed separately.  Inputs rotate over enough copies that the bytes touched
+between two uses of a copy exceed the 126 MB L2, so every step streams from HBM.
+
+Printed on rank 0: one JSON line with the whole-job TFLOP/s, the roofline of the dominant
+kernel (the tcgen05 GEMM, timed live with CUDA events), the online-transform overhead over
+plain MXFP4 (plain quantisation + the same GEMM) and over the GEMM alone, an end-to-end
+figure through the C ABI with host buffers, the oracle's CPU throughput on a bounded
+sample, SM clocks sampled during the timed region, and secondary workloads (decode and
+the Qwen3-32B-shaped down projection).
+
+--impl reference times the CPU oracle (the reference arm of this repository) on a bounded
+sample of the same workload.  With N > 1 GPUs (torchrun), each rank runs an independent
+replica of the layer (the path has no exchange step); value = all ranks' work / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as wls  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def file_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "online_hadamard_b200", "csrc", ent.get("source", ""))
+    if not os.path.exists(src) or file_hash(src) != ent.get("source_hash"):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- setup
+
+
+class Layer:
+    """Folded weights and rotating input copies of one linear on one device."""
+
+    def __init__(self, mq, wl, device, copies=None):
+        self.mq, self.wl, self.dev = mq, wl, device
+        W = wls.make_w(wl)
+        s = wls.make_s(wl, W)
+        x = wls.make_x(wl)
+        footprint = (wl.M * wl.K * 2 + wl.N * wl.K * 0.53125 + wl.M * wl.N * 2 + mq.linear_workspace_bytes(wl.M, wl.K))
+        self.copies = copies or max(2, math.ceil(3 * L2_BYTES / footprint))
+        Wd = W.to(device)
+        sd = s.to(device)
+        self.Wq, self.Ws, self.am, self.x, self.y, self.ws, self.Aq, self.As = [], [], [], [], [], [], [], []
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        for _ in range(self.copies):
+            Wq, Ws, am = mq.macaq_fold_weights(Wd, sd)
+            self.Wq.append(Wq)
+            self.Ws.append(Ws)
+            self.am.append(am)
+        torch.cuda.synchronize(device)
+        self.fold_s = (time.perf_counter() - t0) / self.copies
+        del Wd
+        xd = x.to(device)
+        for _ in range(self.copies):
+            self.x.append(xd.clone())
+            self.y.append(torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=device))
+            self.ws.append(torch.empty(mq.linear_workspace_bytes(wl.M, wl.K), dtype=torch.uint8, device=device))
+            Aq, As = mq.macaq_act_transform_quant(xd, self.am[0])
+            self.Aq.append(Aq)
+            self.As.append(As)
+        self.x_host = x.contiguous().pin_memory()
+        self.y_host = torch.empty(wl.M, wl.N, dtype=torch.bfloat16).pin_memory()
+        torch.cuda.synchronize(device)
+
+    def linear(self, i):
+        c = i % self.copies
+        self.mq.macaq_w4a4_linear(self.x[c], self.am[c], self.Wq[c], self.Ws[c], self.wl.N, y=self.y[c],
+                                  workspace=self.ws[c])
+
+    def gemm(self, i):
+        c = i % self.copies
+        self.mq.macaq_mxfp4_gemm(self.Aq[c], self.As[c], self.Wq[c], self.Ws[c], self.wl.M, self.wl.N, self.wl.K,
+                                 y=self.y[c])
+
+    def plain(self, i):
+        c = i % self.copies
+        self.mq.macaq_act_quant_plain(self.x[c], Aq=self.Aq[c], As=self.As[c])
+        self.mq.macaq_mxfp4_gemm(self.Aq[c], self.As[c], self.Wq[c], self.Ws[c], self.wl.M, self.wl.N, self.wl.K,
+                                 y=self.y[c])
+
+    def transform_only(self, i):
+        c = i % self.copies
+        self.mq.macaq_act_transform_quant(self.x[c], self.am[c], Aq=self.Aq[c], As=self.As[c])
+
+    def e2e(self, i):
+        """Host buffers in, host result out: H2D of x, the linear, D2H of y."""
+        c = i % self.copies
+        self.x[c].copy_(self.x_host, non_blocking=True)
+        self.linear(c)
+        self.y_host.copy_(self.y[c], non_blocking=True)
+
+
+def time_loop(fn, steps, warmup, device):
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        fn(warmup + i)
+    e1.record()
+    torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / steps  # ms per call
+
+
+# --------------------------------------------------------------------------- CPU baseline
+
+
+def cpu_baseline(wl, rows=256, max_rows_time=20.0):
+    """The oracle as it stands, on the host cores: transform + quantise `rows` activation
+    rows and contract them with the folded weights (fold excluded: offline)."""
+    import oracle
+    W = wls.make_w(wl)
+    s = wls.make_s(wl, W)
+    x = wls.make_x(wl)
+    Wq, Ws, a = oracle.fold_weights(W.numpy(), s.numpy())
+    rng = np.random.default_rng(0)
+    idx = np.sort(rng.choice(wl.M, min(rows, wl.M), replace=False))
+    xs = x.float().numpy()[idx]
+    t0 = time.perf_counter()
+    Aq, As = oracle.act_transform_quant(xs, a)
+    oracle.mx_gemm(Aq, As, Wq, Ws)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * len(idx) * wl.N * wl.K
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(idx)} of {wl.M} rows of {wl.name} (transform+quant+fp64 GEMM), {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = wls.LLAMA_UP
+    import oracle
+    W = wls.make_w(wl)
+    s = wls.make_s(wl, W)
+    x = wls.make_x(wl)
+    Wq, Ws, a = oracle.fold_weights(W.numpy(), s.numpy())
+    xs_all = x.float().numpy()
+    rows = 16
+    rng = np.random.default_rng(1)
+    times = []
+    for i in range(args.warmup + args.steps):
+        idx = np.sort(rng.choice(wl.M, rows, replace=False))
+        t0 = time.perf_counter()
+        Aq, As = oracle.act_transform_quant(xs_all[idx], a)
+        oracle.mx_gemm(Aq, As, Wq, Ws)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    dt = sum(times) / len(times)
+    val = 2.0 * rows * wl.N * wl.K / dt / 1e12
+    out = {"impl": "reference", "metric": "W4A4 linear TFLOP/s", "value": val, "unit": "TFLOP/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N},
+           "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": f"{rows} rows of {wl.M} per step"},
+           "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+# --------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    import online_hadamard_b200 as mq
+    mq.load_library()
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+
+    wl = wls.LLAMA_UP
+    layer = Layer(mq, wl, device)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- headline: the fused linear
+    for i in range(args.warmup):
+        layer.linear(i)
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        layer.linear(args.warmup + i)
+    e1.record()
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = world * wl.flops / (ms * 1e-3) / 1e12
+
+    # ---- dominant kernel, the comparators and end to end (same rotation)
+    ms_gemm = time_loop(layer.gemm, args.steps, args.warmup, device)
+    ms_plain = time_loop(layer.plain, args.steps, args.warmup, device)
+    ms_xform = time_loop(layer.transform_only, args.steps, args.warmup, device)
+    e2e_steps = max(3, min(args.steps, 10))
+    ms_e2e = max_over_ranks(time_loop(layer.e2e, e2e_steps, 3, device))
+    gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
+    xform_bytes = wl.M * wl.K * 2 + wl.M * wl.K * (0.5 + 1 / 32) + wl.K * 4
+    traffic = recorded_traffic("mxf4_gemm_128x256:" + wl.name)
+
+    extra = {}
+    if not args.no_extra:
+        extra = secondary(mq, device, peaks, args)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        out = {
+            "metric": "W4A4 linear TFLOP/s (MXFP4 x MXFP4, online scale + FWHT-32 + quant fused ahead of the tcgen05 GEMM)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp4 (e2m1 x e2m1, ue8m0 scales, fp32 accumulate, bf16 out)", "data": "synthetic",
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "parallelism": f"replicas{world}",
+                       "l2": f"inputs rotated over {layer.copies} copies (> 3x L2)"},
+            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_kernel<256,4,false>", "achieved": gemm_tflops,
+                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
+                         "ms_per_launch": ms_gemm},
+            "overhead": {"linear_ms": ms, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
+                         "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
+                         "vs_gemm_only_pct": 100.0 * (ms / ms_gemm - 1.0),
+                         "transform_quant_ms": ms_xform,
+                         "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
+            "e2e": {"value": world * wl.flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+                    "h2d_bytes_per_step": wl.M * wl.K * 2, "d2h_bytes_per_step": wl.M * wl.N * 2},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+            "fold_ms": layer.fold_s * 1e3,
+            "cpu_baseline": cpu,
+            "secondary": extra,
+        }
+        print(json.dumps(out))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def secondary(mq, device, peaks, args):
+    """Decode (HBM-bound) and the Qwen3-32B down projection (tensor-bound)."""
+    res = {}
+    steps = max(10, args.steps // 2)
+    for M in wls.QWEN_DECODE_M:
+        wl = wls.QWEN_UP_DECODE.with_m(M)
+        layer = Layer(mq, wl, device)
+        ms = time_loop(layer.linear, steps, args.warmup, device)
+        ms_plain = time_loop(layer.plain, steps, args.warmup, device)
+        res[f"{wl.name}_M{M}"] = {"ms": ms, "gbs": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9,
+                                   "frac_hbm": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
+        del layer
+        torch.cuda.empty_cache()
+    wl = wls.QWEN_DOWN
+    layer = Layer(mq, wl, device, copies=2)
+    ms = time_loop(layer.linear, steps, args.warmup, device)
+    ms_plain = time_loop(layer.plain, steps, args.warmup, device)
+    ms_gemm = time_loop(layer.gemm, steps, args.warmup, device)
+    t = wl.flops / (ms * 1e-3) / 1e12
+    res[wl.name] = {"ms": ms, "tflops": t, "frac_fp4_peak": t / (peaks["bf16_tflops"] * FP4_OVER_BF16),
+                    "gemm_ms": ms_gemm, "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
+    del layer
+    torch.cuda.empty_cache()
+    return res
+
+
+if __name__ == "__main__":
+    main()

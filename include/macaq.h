@@ -1,0 +1,150 @@
+/*
+ * macaq.h -- C ABI of libmacaq: the inference hot path of MACaQ's layer-local MXFP4 W4A4
+ * linear layer on NVIDIA B200 (sm_100a).
+ *
+ * Method: "MACaQ: Fast, Model Agnostic Calibrated Quantization for Low-Precision Weights
+ * and Activations" (arXiv 2611.10649), Abstract: every linear layer is treated on its
+ * own; a per-channel scale and a block-Hadamard transform are applied online to the
+ * layer's activations while the corresponding inverse transforms are absorbed into the
+ * layer's weights; weights and activations are MXFP4 (W4A4), the weights rounded to
+ * nearest.  The pages leave the details open; this library fixes them as follows.
+ *
+ *   Notation.  x is bf16 [M][K] row-major, W is fp32 [N][K] row-major (y = x W^T, the
+ *   nn.Linear layout), s is fp32 [K] with s_k > 0 finite.  c = 1/sqrt(32).
+ *   Block-Hadamard: blocks of b = 32 consecutive k, Sylvester order
+ *   H[i][j] = (-1)^popcount(i&j), applied unnormalised; its 1/sqrt(32) goes into one fp32
+ *   multiplier per channel:  act_mult[k] = fl32(c / s_k),  w_mult[k] = fl32(s_k * c).
+ *   Activations are divided by s, weights multiplied by s, so that
+ *   (x diag(1/s) H/sqrt32)(W diag(s) H/sqrt32)^T = x W^T.
+ *   Transform (fp32, one canonical order): u_k = fl32(x_k * mult_k), then butterfly stages
+ *   h = 1, 2, 4, 8, 16 replacing (u_i, u_{i+h}) by (u_i + u_{i+h}, u_i - u_{i+h}).
+ *   MXFP4 (OCP Microscaling v1.0): per 32-block, E8M0 scale byte e = max(E(amax) - 2, 0)
+ *   where E(amax) is the biased fp32 exponent of the block's largest |v| (e never reaches
+ *   0xFF); element code = (sign << 3) | index of v * 2^(127-e) rounded to the nearest of
+ *   {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even index, saturating at 6; the IEEE sign
+ *   is kept, so a negative value rounding to zero is code 0x8.
+ *
+ * Data layouts (all sizes in bytes, all buffers caller-allocated and caller-owned):
+ *
+ *   MXFP4 codes   uint8 [rows][K/2]: element k of a row sits in byte k/2, low nibble
+ *                 when k is even.
+ *   E8M0 scales   "MMA tile layout": uint8, macaq_scale_bytes(rows, K) bytes.  Rows are
+ *                 padded to a multiple of 128 and the K/32 blocks of a row to a multiple
+ *                 of 8; the byte of (row r, block kb) is at macaq_scale_offset(r, kb, K) =
+ *                   ((r/128) * (KBp/4) + kb/4) * 512 + (r%32)*16 + ((r/32)%4)*4 + kb%4,
+ *                 KBp = 8 * ceil(K/256).  Each 512-byte atom holds 4 blocks of 128 rows in
+ *                 the order the tensor cores' scale-factor copy expects.  Writers fill the
+ *                 padded blocks of real rows with 0; bytes of padded rows are never used
+ *                 for a stored output and may hold anything.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers on the current CUDA device, 16-byte aligned;
+ *     otherwise MACAQ_EALIGN.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - M, N >= 1, 32 <= K, K % 32 == 0, and M, N, K < 2^31; otherwise MACAQ_ESHAPE.
+ *   - The calls validate, enqueue kernels on `stream` and return; the return value is the
+ *     validation/launch status.  Errors of the asynchronous work surface at the next
+ *     synchronisation; a device-side wait that gives up (it never should) sets a flag
+ *     that macaq_device_status() reports.  No call allocates device memory, except as
+ *     stated for macaq_fold_weights (none) -- scratch is passed in by the caller.
+ *   - Non-finite activations or weights are out of scope (codes are then unspecified).
+ */
+#ifndef MACAQ_H_
+#define MACAQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MACAQ_OK = 0,
+    MACAQ_EINVAL = -1,     /* null pointer, non-finite or non-positive s, bad flag */
+    MACAQ_ESHAPE = -2,     /* M, N, K out of range or K % 32 != 0 */
+    MACAQ_EALIGN = -3,     /* a pointer is not 16-byte aligned */
+    MACAQ_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed */
+    MACAQ_ETIMEOUT = -5,   /* a bounded device-side wait gave up (see macaq_device_status) */
+    MACAQ_EWORKSPACE = -6  /* workspace smaller than the call needs */
+} macaq_status;
+
+/* Human-readable name of a status code (static storage). */
+const char* macaq_status_str(int status);
+
+/* Bytes of an E8M0 scale buffer in the MMA tile layout for `rows` x K elements
+ * (0 on invalid arguments). */
+size_t macaq_scale_bytes(int64_t rows, int64_t K);
+
+/* Offset of the scale byte of (row r, 32-block kb) in that buffer (-1 if out of range). */
+int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
+
+/* Bytes of scratch macaq_w4a4_linear needs for M x K activations: their MXFP4 codes
+ * (M*K/2, rounded up to 256) plus scales (macaq_scale_bytes(M, K)). */
+size_t macaq_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * macaq_fold_weights -- offline weight preparation (Abstract: "absorbing the corresponding
+ * inverse transforms into its weights"; weights quantised round-to-nearest).
+ *   W        in   fp32 [N][K]
+ *   s        in   fp32 [K], every s_k finite and > 0 (else MACAQ_EINVAL, nothing written)
+ *   Wq       out  MXFP4 codes [N][K/2] of W' = W diag(s) H_bd / sqrt(32)
+ *   Ws       out  E8M0 scales of W', MMA tile layout, macaq_scale_bytes(N, K) bytes
+ *   act_mult out  fp32 [K], fl32(c / s_k): the online activation multiplier
+ * This offline call copies s to the host to validate it and therefore synchronises
+ * `stream`; the hot-path calls below never synchronise.
+ */
+int macaq_fold_weights(const float* W, int64_t N, int64_t K, const float* s, uint8_t* Wq,
+                       uint8_t* Ws, float* act_mult, void* stream);
+
+/*
+ * macaq_act_transform_quant -- the online activation transform (Abstract: "a per-channel
+ * scale and a block-Hadamard transform online to each layer's activations") followed by
+ * MXFP4 quantisation (the A4 of W4A4).
+ *   x        in   bf16 bit patterns [M][K]
+ *   act_mult in   fp32 [K] (from macaq_fold_weights)
+ *   Aq       out  MXFP4 codes [M][K/2]
+ *   As       out  E8M0 scales, MMA tile layout, macaq_scale_bytes(M, K) bytes
+ */
+int macaq_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
+                              uint8_t* Aq, uint8_t* As, void* stream);
+
+/*
+ * macaq_w4a4_linear -- the layer's forward pass, y = x W^T computed as
+ * MXFP4(x diag(act_mult) H) . MXFP4(W')^T (Abstract; the 2.3% end-to-end overhead over
+ * plain MXFP4 quoted there is for this online transform): the activation transform and
+ * quantisation run as the GEMM's prologue, the block-scaled MXFP4 x MXFP4 contraction
+ * runs on the tensor cores with fp32 accumulation, and y is rounded to bf16 (RNE).
+ *   x         in   bf16 [M][K];  act_mult in fp32 [K]
+ *   Wq, Ws    in   folded weights from macaq_fold_weights (N rows)
+ *   y         out  bf16 [M][N]
+ *   workspace in   scratch of at least macaq_linear_workspace_bytes(M, K) bytes
+ *                  (MACAQ_EWORKSPACE otherwise); its contents on return are unspecified
+ *                  and calls sharing one workspace must be stream-ordered.
+ */
+int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
+                      const uint8_t* Wq, const uint8_t* Ws, int64_t N, uint16_t* y,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Baselines and building blocks (not part of the method; used to measure the overhead of
+ * the online transform against "pure MXFP4", Abstract).
+ *
+ * macaq_act_quant_plain: MXFP4 quantisation of x with no scale and no transform.
+ * macaq_mxfp4_gemm: y = dec(A) dec(W)^T for already-quantised operands, fp32 accumulate;
+ *   y is bf16 [M][N] (y_is_fp32 = 0) or fp32 [M][N] (y_is_fp32 = 1).
+ */
+int macaq_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
+                          void* stream);
+int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
+                     const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32,
+                     void* stream);
+
+/* Sticky device-side status of the current device: MACAQ_OK, or MACAQ_ETIMEOUT once a
+ * bounded wait inside a kernel gave up.  Synchronises the device.  `clear` != 0 resets it. */
+int macaq_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MACAQ_H_ */

@@ -1,0 +1,200 @@
+"""Python binding of libmacaq: the MACaQ MXFP4 W4A4 linear layer on B200 (sm_100a).
+
+Argument marshalling only: every function below checks tensor placement, dtype and
+contiguity, allocates outputs with torch when the caller does not pass them, and calls the
+C entry point of the same name in ``_build/libmacaq.so`` on the current CUDA stream.  All
+arithmetic runs in the library's CUDA kernels; there is no CPU or PyTorch fallback -- if
+the library cannot be loaded, every call raises.
+
+Method: "MACaQ: Fast, Model Agnostic Calibrated Quantization for Low-Precision Weights and
+Activations", Abstract (per-channel scale and block-Hadamard applied online to the
+activations, inverse transforms absorbed into the weights, MXFP4 W4A4).  Layouts and
+conventions are documented in include/macaq.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build_mod
+
+__all__ = [
+    "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes",
+    "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
+    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status", "status_str",
+    "EXPORTED_SYMBOLS",
+]
+
+# Every symbol include/macaq.h declares.
+EXPORTED_SYMBOLS = (
+    "macaq_status_str", "macaq_scale_bytes", "macaq_scale_offset", "macaq_linear_workspace_bytes",
+    "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
+    "macaq_act_quant_plain", "macaq_mxfp4_gemm", "macaq_device_status",
+)
+
+MACAQ_OK = 0
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MacaqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_str(status)} ({status})")
+        self.status = status
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load (building first if absent) libmacaq.so and declare its C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        lib_path = path or _build_mod.LIB_PATH
+        if path is None and not os.path.exists(lib_path):
+            _build_mod.build()
+        lib = ctypes.CDLL(lib_path)
+        p, i64, sz, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+        lib.macaq_status_str.argtypes = [i32]
+        lib.macaq_status_str.restype = ctypes.c_char_p
+        lib.macaq_scale_bytes.argtypes = [i64, i64]
+        lib.macaq_scale_bytes.restype = sz
+        lib.macaq_scale_offset.argtypes = [i64, i64, i64]
+        lib.macaq_scale_offset.restype = i64
+        lib.macaq_linear_workspace_bytes.argtypes = [i64, i64]
+        lib.macaq_linear_workspace_bytes.restype = sz
+        lib.macaq_fold_weights.argtypes = [p, i64, i64, p, p, p, p, p]
+        lib.macaq_act_transform_quant.argtypes = [p, i64, i64, p, p, p, p]
+        lib.macaq_act_quant_plain.argtypes = [p, i64, i64, p, p, p]
+        lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p]
+        lib.macaq_w4a4_linear.argtypes = [p, i64, i64, p, p, p, i64, p, p, sz, p]
+        lib.macaq_device_status.argtypes = [i32]
+        for name in ("macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
+                     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status"):
+            getattr(lib, name).restype = i32
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_str(status: int) -> str:
+    return load_library().macaq_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MACAQ_OK:
+        raise MacaqError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def scale_bytes(rows: int, K: int) -> int:
+    """Size of an E8M0 scale buffer in the MMA tile layout (include/macaq.h)."""
+    return int(load_library().macaq_scale_bytes(rows, K))
+
+
+def scale_offset(r: int, kb: int, K: int) -> int:
+    return int(load_library().macaq_scale_offset(r, kb, K))
+
+
+def linear_workspace_bytes(M: int, K: int) -> int:
+    return int(load_library().macaq_linear_workspace_bytes(M, K))
+
+
+def macaq_fold_weights(W: torch.Tensor, s: torch.Tensor, Wq=None, Ws=None, act_mult=None, stream=None):
+    """Fold diag(s) H/sqrt(32) into W (fp32 [N, K]) and RTN-quantise: (Wq, Ws, act_mult)."""
+    N, K = W.shape
+    _need(W, "W", torch.float32)
+    _need(s, "s", torch.float32, (K,))
+    dev = W.device
+    Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev) if Wq is None else Wq
+    Ws = torch.empty(max(scale_bytes(N, K), 1), dtype=torch.uint8, device=dev) if Ws is None else Ws
+    act_mult = torch.empty(K, dtype=torch.float32, device=dev) if act_mult is None else act_mult
+    _check(load_library().macaq_fold_weights(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(Ws), _ptr(act_mult),
+                                             _stream(stream)), "macaq_fold_weights")
+    return Wq, Ws, act_mult
+
+
+def macaq_act_transform_quant(x: torch.Tensor, act_mult: torch.Tensor, Aq=None, As=None, stream=None):
+    """Scale, FWHT-32 and MXFP4-quantise bf16 activations [M, K]: (Aq, As)."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(act_mult, "act_mult", torch.float32, (K,))
+    dev = x.device
+    Aq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Aq is None else Aq
+    As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
+    _check(load_library().macaq_act_transform_quant(_ptr(x), M, K, _ptr(act_mult), _ptr(Aq), _ptr(As),
+                                                    _stream(stream)), "macaq_act_transform_quant")
+    return Aq, As
+
+
+def macaq_act_quant_plain(x: torch.Tensor, Aq=None, As=None, stream=None):
+    """Plain MXFP4 quantisation of bf16 activations (no scale, no transform): (Aq, As)."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    Aq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Aq is None else Aq
+    As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
+    _check(load_library().macaq_act_quant_plain(_ptr(x), M, K, _ptr(Aq), _ptr(As), _stream(stream)),
+           "macaq_act_quant_plain")
+    return Aq, As
+
+
+def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: bool = False, stream=None):
+    """y = dec(A) dec(W)^T from MXFP4 operands; bf16 (default) or fp32 [M, N]."""
+    _need(Aq, "Aq", torch.uint8, (M, K // 2))
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(As, "As", torch.uint8)
+    _need(Ws, "Ws", torch.uint8)
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    y = torch.empty(M, N, dtype=dt, device=Aq.device) if y is None else y
+    _need(y, "y", dt, (M, N))
+    _check(load_library().macaq_mxfp4_gemm(_ptr(Aq), _ptr(As), M, _ptr(Wq), _ptr(Ws), N, K, _ptr(y),
+                                           1 if out_fp32 else 0, _stream(stream)), "macaq_mxfp4_gemm")
+    return y
+
+
+def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+                      y=None, workspace=None, stream=None):
+    """y = x W^T through the online transform, MXFP4 quantisation and the W4A4 GEMM (bf16 [M, N])."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(act_mult, "act_mult", torch.float32, (K,))
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(Ws, "Ws", torch.uint8)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    need = linear_workspace_bytes(M, K)
+    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8)
+    _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+                                            _ptr(workspace), workspace.numel(), _stream(stream)),
+           "macaq_w4a4_linear")
+    return y
+
+
+def macaq_device_status(clear: bool = False) -> int:
+    """MACAQ_OK, or MACAQ_ETIMEOUT if a bounded device-side wait gave up (synchronises)."""
+    return int(load_library().macaq_device_status(1 if clear else 0))

@@ -1,0 +1,64 @@
+// api.cu -- status strings, buffer-size helpers and the device status flag of libmacaq.
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace macaq {
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+}  // namespace macaq
+
+using namespace macaq;
+
+extern "C" const char* macaq_status_str(int status) {
+    switch (status) {
+        case MACAQ_OK: return "MACAQ_OK";
+        case MACAQ_EINVAL: return "MACAQ_EINVAL: null pointer or invalid value";
+        case MACAQ_ESHAPE: return "MACAQ_ESHAPE: M, N, K out of range or K not a multiple of 32";
+        case MACAQ_EALIGN: return "MACAQ_EALIGN: pointer not 16-byte aligned";
+        case MACAQ_ECUDA: return "MACAQ_ECUDA: CUDA runtime or launch failure";
+        case MACAQ_ETIMEOUT: return "MACAQ_ETIMEOUT: a bounded device-side wait gave up";
+        case MACAQ_EWORKSPACE: return "MACAQ_EWORKSPACE: workspace too small";
+        default: return "MACAQ: unknown status";
+    }
+}
+
+extern "C" size_t macaq_scale_bytes(int64_t rows, int64_t K) {
+    if (check_shape(rows, K) != MACAQ_OK) return 0;
+    return static_cast<size_t>(scale_bytes(rows, K));
+}
+
+extern "C" int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K) {
+    if (r < 0 || r > kMaxDim || K < kBlock || K > kMaxDim || K % kBlock != 0) return -1;
+    if (kb < 0 || kb >= padded_blocks(K)) return -1;
+    return scale_offset(r, kb, padded_blocks(K));
+}
+
+extern "C" size_t macaq_linear_workspace_bytes(int64_t M, int64_t K) {
+    if (check_shape(M, K) != MACAQ_OK) return 0;
+    const int64_t codes = ((M * (K / 2) + 255) / 256) * 256;
+    return static_cast<size_t>(codes + scale_bytes(M, K));
+}
+
+extern "C" int macaq_device_status(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MACAQ_ECUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MACAQ_ECUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MACAQ_ECUDA;
+    }
+    return v == 0 ? MACAQ_OK : MACAQ_ETIMEOUT;
+}

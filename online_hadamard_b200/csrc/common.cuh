@@ -1,0 +1,46 @@
+// common.cuh -- shapes, the E8M0 scale tile layout and host-side validation shared by the
+// library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "macaq.h"
+
+namespace macaq {
+
+constexpr int64_t kBlock = 32;          // MX block = Hadamard block (elements along K)
+constexpr int64_t kMaxDim = 0x7FFFFFFF;  // M, N, K < 2^31
+
+// Scale blocks per row, padded so every 256-element K tile owns two full 512-byte atoms.
+__host__ __device__ __forceinline__ int64_t padded_blocks(int64_t K) {
+    return ((K + 255) / 256) * 8;
+}
+
+// Byte offset of the E8M0 scale of (row r, 32-block kb) in the MMA tile layout: 512-byte
+// atoms of 128 rows x 4 blocks, atom (r/128, kb/4) at ((r/128) * KBp/4 + kb/4) * 512,
+// inside it row r at (r%32)*16 + ((r/32)%4)*4 and block kb at kb%4.
+__host__ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t kb, int64_t kbp) {
+    return ((r >> 7) * (kbp >> 2) + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+__host__ __device__ __forceinline__ int64_t scale_bytes(int64_t rows, int64_t K) {
+    return ((rows + 127) / 128) * 128 * padded_blocks(K);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int check_shape(int64_t rows, int64_t K) {
+    if (rows < 1 || rows > kMaxDim || K < kBlock || K > kMaxDim || K % kBlock != 0) return MACAQ_ESHAPE;
+    return MACAQ_OK;
+}
+
+inline int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ECUDA;
+}
+
+// Number of SMs of the current device (cached per device ordinal).
+int sm_count();
+
+}  // namespace macaq

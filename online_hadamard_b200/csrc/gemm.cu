@@ -1,0 +1,423 @@
+// gemm.cu -- block-scaled MXFP4 x MXFP4 GEMM on the sm_100a tensor cores, and the fused
+// MACaQ W4A4 linear layer built on it.
+//
+// y[m][n] = sum_b 2^(eA[m][b]-127) 2^(eW[n][b]-127) sum_{i<32} e2m1(A[m][32b+i]) e2m1(W[n][32b+i])
+// with fp32 accumulation (tcgen05.mma kind::mxf4, E8M0 scales, one per 32 elements), y in
+// bf16 (round to nearest even) or fp32.  "MACaQ: Fast, Model Agnostic Calibrated
+// Quantization for Low-Precision Weights and Activations", Abstract: MXFP4 W4A4 -- both
+// operands of every linear layer are MXFP4; the W4A4 matmul is the dense contraction the
+// method runs at inference time.
+//
+// Kernel design (one CTA per SM, persistent over output tiles):
+//   tile       128 rows of the "P" operand (MMA M) x BN rows of the "Q" operand (MMA N),
+//              K consumed 256 elements (128 bytes of codes per row) per pipeline stage.
+//              P = A, Q = W for large M;  P = W, Q = A ("swap-AB") for small M, so the
+//              weight rows fill the 128-row MMA and a few tokens form a narrow N.
+//   warp 0     producer: TMA (128-byte swizzle) loads of both code tiles and linear bulk
+//              copies of the matching 512-byte scale atoms into a STAGES-deep ring.
+//   warp 1     allocates tensor memory; one lane issues, per stage, tcgen05.cp of the
+//              scale atoms into TMEM and four tcgen05.mma (K = 64 each), then commits the
+//              stage back to the producer and, per tile, the accumulator to the epilogue.
+//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads TMEM lanes of
+//              sub-partition w % 4), conversion, and stores of y.
+//   Accumulators are double-buffered in TMEM when BN <= 128 so the epilogue of one tile
+//   overlaps the mainloop of the next.  All waits are bounded (see sm100.cuh).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace macaq {
+
+int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
+                               uint8_t* Aq, uint8_t* As, cudaStream_t stream);
+
+constexpr int kBM = 128;           // MMA M
+constexpr int kStageK = 256;       // K elements per stage
+constexpr int kStageKBytes = 128;  // code bytes per row per stage
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct TileCfg {
+    static constexpr int kQBlocks = (BN + 127) / 128;  // 128-row scale atoms on the Q side
+    static constexpr int kPBytes = kBM * kStageKBytes;
+    static constexpr int kQBytes = BN * kStageKBytes;
+    static constexpr int kSFPBytes = 1024;             // 2 atoms: 128 rows x 8 blocks
+    static constexpr int kSFQBytes = 1024 * kQBlocks;
+    static constexpr int kStageBytes = kPBytes + kQBytes + kSFPBytes + kSFQBytes;
+    static constexpr int kNumAcc = BN <= 128 ? 2 : 1;
+    static constexpr int kAccStride = ((BN + 31) / 32) * 32;
+    static constexpr int kSFPCol = kNumAcc * kAccStride;           // 2 groups x 4 columns
+    static constexpr int kSFQCol = kSFPCol + 8;
+    static constexpr int kSFQColsPerGroup = 4 * kQBlocks;
+    static constexpr int kColsUsed = kSFQCol + 2 * kSFQColsPerGroup;
+    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                   : kColsUsed <= 256 ? 256 : 512;
+    static_assert(kColsUsed <= 512, "tensor memory budget");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
+};
+
+struct GemmParams {
+    const uint8_t* sf_p;  // scales of P, MMA tile layout
+    const uint8_t* sf_q;  // scales of Q
+    int64_t p_rows, q_rows, K, kbp;
+    void* y;
+    int64_t ldy;          // elements per row of y
+    int y_fp32;
+    int num_p_tiles, num_q_tiles, num_k_tiles, q_row_blocks;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Store CH accumulator columns [qc, qc+CH) of P-row `prow`.
+template <int CH, bool SWAP>
+__device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow, int64_t qc,
+                                            const uint32_t* r) {
+    if (prow >= prm.p_rows) return;
+    if constexpr (!SWAP) {
+        const int64_t base = prow * prm.ldy + qc;
+        const bool full = qc + CH <= prm.q_rows;
+        if (prm.y_fp32) {
+            float* y = static_cast<float*>(prm.y) + base;
+            if (full && (prm.ldy % 4) == 0) {
+#pragma unroll
+                for (int j = 0; j < CH; j += 4)
+                    *reinterpret_cast<uint4*>(y + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+            } else {
+                for (int j = 0; j < CH && qc + j < prm.q_rows; ++j) y[j] = __uint_as_float(r[j]);
+            }
+        } else {
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(prm.y) + base;
+            if (full && (prm.ldy % 8) == 0) {
+#pragma unroll
+                for (int j = 0; j < CH; j += 8)
+                    *reinterpret_cast<uint4*>(y + j) =
+                        make_uint4(pack_bf16x2(r[j], r[j + 1]), pack_bf16x2(r[j + 2], r[j + 3]),
+                                   pack_bf16x2(r[j + 4], r[j + 5]), pack_bf16x2(r[j + 6], r[j + 7]));
+            } else {
+                for (int j = 0; j < CH && qc + j < prm.q_rows; ++j) y[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+            }
+        }
+    } else {
+        // accumulator row = output column (feature), accumulator column = output row (token)
+        if (prm.y_fp32) {
+            float* y = static_cast<float*>(prm.y);
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+                if (qc + j < prm.q_rows) y[(qc + j) * prm.ldy + prow] = __uint_as_float(r[j]);
+        } else {
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(prm.y);
+#pragma unroll
+            for (int j = 0; j < CH; ++j)
+                if (qc + j < prm.q_rows) y[(qc + j) * prm.ldy + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
+    }
+}
+
+template <int BN, int STAGES, bool SWAP>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
+                     const GemmParams prm) {
+    using Cfg = TileCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 128);
+        }
+        fence_mbar_init();
+        prefetch_tmap(&tmap_p);
+        prefetch_tmap(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_tiles = prm.num_p_tiles * prm.num_q_tiles;
+    int abort = 0;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------------- producer
+            griddep_wait();  // operands may come from the kernel launched just before
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !abort; tile += gridDim.x) {
+                const int pt = tile % prm.num_p_tiles;
+                const int qt = tile / prm.num_p_tiles;
+                const uint8_t* sfp = prm.sf_p + static_cast<int64_t>(pt) * (prm.kbp / 4) * 512;
+                for (int kt = 0; kt < prm.num_k_tiles; ++kt) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
+                    uint8_t* sb = smem + stage * Cfg::kStageBytes;
+                    mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
+                    tma_load_2d(sb, &tmap_p, kt * kStageKBytes, pt * kBM, &full[stage]);
+                    tma_load_2d(sb + Cfg::kPBytes, &tmap_q, kt * kStageKBytes, qt * BN, &full[stage]);
+                    bulk_load(sb + Cfg::kPBytes + Cfg::kQBytes, sfp + kt * 1024, 1024, &full[stage]);
+#pragma unroll
+                    for (int i = 0; i < Cfg::kQBlocks; ++i) {
+                        int qb = (qt * BN) / 128 + i;
+                        if (qb >= prm.q_row_blocks) qb = prm.q_row_blocks - 1;  // rows past the end: masked
+                        bulk_load(sb + Cfg::kPBytes + Cfg::kQBytes + Cfg::kSFPBytes + 1024 * i,
+                                  prm.sf_q + static_cast<int64_t>(qb) * (prm.kbp / 4) * 512 + kt * 1024, 1024,
+                                  &full[stage]);
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // -------------------------------------------------------------- MMA issuer
+            // instruction descriptor: E2M1 x E2M1 (kind::mxf4), UE8M0 scales, K-major A/B
+            const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) | (1u << 23) |
+                                   (static_cast<uint32_t>(kBM >> 4) << 24);
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !abort; tile += gridDim.x) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * Cfg::kAccStride;
+                for (int kt = 0; kt < prm.num_k_tiles; ++kt) {
+                    if (!mbar_wait(&full[stage], phase, &abort)) break;
+                    tc_fence_after();
+                    const uint32_t sp = smem_u32(smem + stage * Cfg::kStageBytes);
+                    const uint32_t sq = sp + Cfg::kPBytes;
+                    const uint32_t ssfp = sq + Cfg::kQBytes;
+                    const uint32_t ssfq = ssfp + Cfg::kSFPBytes;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        tc_cp_sf(tmem_base + Cfg::kSFPCol + 4 * g, desc_sf(ssfp + 512 * g));
+#pragma unroll
+                        for (int i = 0; i < Cfg::kQBlocks; ++i)
+                            tc_cp_sf(tmem_base + Cfg::kSFQCol + Cfg::kSFQColsPerGroup * g + 4 * i,
+                                     desc_sf(ssfq + 1024 * i + 512 * g));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t g = j >> 1;
+                        const uint32_t id = (j & 1) * 2;  // byte of the scale word: blocks 2j%4, 2j%4+1
+                        const uint32_t sfa = (tmem_base + Cfg::kSFPCol + 4 * g) | (id << 30);
+                        const uint32_t sfb = (tmem_base + Cfg::kSFQCol + Cfg::kSFQColsPerGroup * g) | (id << 30);
+                        tc_mma_mxf4(d_tmem, desc_sw128(sp + 32 * j), desc_sw128(sq + 32 * j),
+                                    idesc | (id << 29) | (id << 4), sfa, sfb, (kt | j) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                tc_commit(&acc_full[acc]);
+                if (++acc == Cfg::kNumAcc) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int sub = warp & 3;  // TMEM sub-partition this warp may read
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && !abort; tile += gridDim.x) {
+            const int pt = tile % prm.num_p_tiles;
+            const int qt = tile / prm.num_p_tiles;
+            if (!mbar_wait(&acc_full[acc], acc_phase, &abort)) break;
+            tc_fence_after();
+            const int64_t prow = static_cast<int64_t>(pt) * kBM + sub * 32 + lane;
+            const uint32_t tbase = tmem_base + acc * Cfg::kAccStride + (static_cast<uint32_t>(sub * 32) << 16);
+            if constexpr (BN % 32 == 0) {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + c, r);
+                    tmem_ld_wait();
+                    store_chunk<32, SWAP>(prm, prow, static_cast<int64_t>(qt) * BN + c, r);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tbase + c, r);
+                    tmem_ld_wait();
+                    store_chunk<16, SWAP>(prm, prow, static_cast<int64_t>(qt) * BN + c, r);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);
+            if (++acc == Cfg::kNumAcc) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+// --------------------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of an MXFP4 code matrix [rows][K/2] bytes: boxes of box_rows x 128 bytes,
+// 128-byte swizzle, zero fill past the edges (ragged M, N and K tails).
+static bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(kStageKBytes), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct GemmOperands {
+    const uint8_t *pq, *ps, *qq, *qs;
+    int64_t p_rows, q_rows, K;
+    void* y;
+    int64_t ldy;
+    int y_fp32;
+};
+
+template <int BN, int STAGES, bool SWAP>
+static int launch_gemm(const GemmOperands& op, cudaStream_t stream, bool pdl) {
+    using Cfg = TileCfg<BN>;
+    CUtensorMap mp, mq;
+    if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, op.q_rows, op.K, BN))
+        return MACAQ_ECUDA;
+    GemmParams prm;
+    prm.sf_p = op.ps;
+    prm.sf_q = op.qs;
+    prm.p_rows = op.p_rows;
+    prm.q_rows = op.q_rows;
+    prm.K = op.K;
+    prm.kbp = padded_blocks(op.K);
+    prm.y = op.y;
+    prm.ldy = op.ldy;
+    prm.y_fp32 = op.y_fp32;
+    prm.num_p_tiles = static_cast<int>((op.p_rows + kBM - 1) / kBM);
+    prm.num_q_tiles = static_cast<int>((op.q_rows + BN - 1) / BN);
+    prm.num_k_tiles = static_cast<int>((op.K + kStageK - 1) / kStageK);
+    prm.q_row_blocks = static_cast<int>((op.q_rows + 127) / 128);
+
+    auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP>;
+    const int smem = STAGES * Cfg::kStageBytes + (2 * STAGES + 4) * 8 + 16 + 1024;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return MACAQ_ECUDA;
+    int occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kGemmThreads, smem) != cudaSuccess || occ < 1)
+        occ = 1;
+    if (occ * Cfg::kTmemCols > 512) occ = 512 / Cfg::kTmemCols;
+    const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
+    int64_t grid = static_cast<int64_t>(sm_count()) * occ;
+    if (grid > tiles) grid = tiles;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, mp, mq, prm) != cudaSuccess) return MACAQ_ECUDA;
+    return launch_status();
+}
+
+// y[M][N] = dec(A) dec(W)^T.  Small M runs swap-AB (weights on the MMA M side).
+int run_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq, const uint8_t* Ws,
+                   int64_t N, int64_t K, void* y, int y_fp32, cudaStream_t stream, bool pdl) {
+    if (M <= 128) {
+        GemmOperands op{Wq, Ws, Aq, As, N, M, K, y, N, y_fp32};
+        if (M <= 16) return launch_gemm<16, 5, true>(op, stream, pdl);
+        if (M <= 32) return launch_gemm<32, 4, true>(op, stream, pdl);
+        if (M <= 64) return launch_gemm<64, 4, true>(op, stream, pdl);
+        return launch_gemm<128, 6, true>(op, stream, pdl);
+    }
+    GemmOperands op{Aq, As, Wq, Ws, M, N, K, y, N, y_fp32};
+    return launch_gemm<256, 4, false>(op, stream, pdl);
+}
+
+}  // namespace macaq
+
+using namespace macaq;
+
+extern "C" int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
+                                const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32, void* stream) {
+    if (!Aq || !As || !Wq || !Ws || !y) return MACAQ_EINVAL;
+    if (y_is_fp32 != 0 && y_is_fp32 != 1) return MACAQ_EINVAL;
+    if (int st = check_shape(M, K)) return st;
+    if (int st = check_shape(N, K)) return st;
+    if (!aligned16(Aq) || !aligned16(As) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y)) return MACAQ_EALIGN;
+    return run_mxfp4_gemm(Aq, As, M, Wq, Ws, N, K, y, y_is_fp32, static_cast<cudaStream_t>(stream), false);
+}
+
+extern "C" int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult, const uint8_t* Wq,
+                                 const uint8_t* Ws, int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+    if (!x || !act_mult || !Wq || !Ws || !y || !workspace) return MACAQ_EINVAL;
+    if (int st = check_shape(M, K)) return st;
+    if (int st = check_shape(N, K)) return st;
+    if (!aligned16(x) || !aligned16(act_mult) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y) ||
+        !aligned16(workspace))
+        return MACAQ_EALIGN;
+    if (workspace_bytes < macaq_linear_workspace_bytes(M, K)) return MACAQ_EWORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* Aq = static_cast<uint8_t*>(workspace);
+    uint8_t* As = Aq + ((M * (K / 2) + 255) / 256) * 256;
+    if (int rc = launch_act_transform_quant(x, M, K, act_mult, Aq, As, st)) return rc;
+    return run_mxfp4_gemm(Aq, As, M, Wq, Ws, N, K, y, 0, st, true);
+}

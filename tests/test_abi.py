@@ -1,0 +1,92 @@
+"""The C ABI: the library loads, exports every symbol include/macaq.h declares, and its
+host-side helpers and argument validation behave as documented (no GPU needed: every
+case here returns before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import online_hadamard_b200 as mq
+from tests import layout
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "macaq.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(macaq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_symbols() == sorted(mq.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = mq.load_library()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    # and through the dynamic symbol table directly
+    raw = ctypes.CDLL(mq._build_mod.LIB_PATH)
+    for name in declared_symbols():
+        assert ctypes.cast(getattr(raw, name), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert mq.status_str(code).startswith("MACAQ")
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (16, 256), (129, 96), (2048, 4096), (300, 25600), (5, 800)])
+def test_scale_layout_helpers_match_documentation(rows, K):
+    assert mq.scale_bytes(rows, K) == layout.scale_bytes(rows, K)
+    idx = layout.scale_index(rows, K, layout.padded_blocks(K))
+    rng = np.random.default_rng(rows + K)
+    for _ in range(50):
+        r = int(rng.integers(rows))
+        kb = int(rng.integers(layout.padded_blocks(K)))
+        assert mq.scale_offset(r, kb, K) == idx[r, kb]
+    # the map is a bijection onto the buffer when rows fill whole 128-row atoms
+    full = layout.scale_index(((rows + 127) // 128) * 128, K, layout.padded_blocks(K))
+    assert np.array_equal(np.sort(full.ravel()), np.arange(layout.scale_bytes(rows, K)))
+
+
+def test_size_helpers_reject_bad_shapes():
+    assert mq.scale_bytes(0, 256) == 0
+    assert mq.scale_bytes(4, 48) == 0
+    assert mq.scale_offset(0, 8, 256) == -1
+    assert mq.linear_workspace_bytes(16, 33) == 0
+    ws = mq.linear_workspace_bytes(16, 256)
+    assert ws == 256 * ((16 * 128 + 255) // 256) + layout.scale_bytes(16, 256)
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
+MIS = 0x10008
+
+
+def _call(name, *args):
+    lib = mq.load_library()
+    return getattr(lib, name)(*args)
+
+
+def test_validation_null_shape_alignment():
+    P = ctypes.c_void_p
+    # null pointers
+    assert _call("macaq_act_transform_quant", None, 4, 64, P(FAKE), P(FAKE), P(FAKE), None) == -1
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, None, 0, None) == -1
+    # shapes
+    assert _call("macaq_act_transform_quant", P(FAKE), 4, 48, P(FAKE), P(FAKE), P(FAKE), None) == -2
+    assert _call("macaq_act_quant_plain", P(FAKE), 0, 64, P(FAKE), P(FAKE), None) == -2
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 0, 64, P(FAKE), 0, None) == -2
+    assert _call("macaq_fold_weights", P(FAKE), 8, 16, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None) == -2
+    # alignment
+    assert _call("macaq_act_transform_quant", P(MIS), 4, 64, P(FAKE), P(FAKE), P(FAKE), None) == -3
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(MIS), 0, None) == -3
+    # bad flag
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(FAKE), 2, None) == -1
+    # workspace too small
+    need = mq.linear_workspace_bytes(4, 64)
+    assert _call("macaq_w4a4_linear", P(FAKE), 4, 64, P(FAKE), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE),
+                 need - 1, None) == -6

@@ -1,0 +1,77 @@
+"""End-to-end parity of the W4A4 linear layer (fold + online transform + GEMM) against the
+oracle run on its OWN codes: the oracle folds W, transforms and quantises x and contracts
+in fp64 ("MACaQ", Abstract).  Because codes and scales are bit-exact, the GPU's bf16 y
+must match bf16(y_oracle) within the GEMM tolerance.  The W4A4 error against the
+unquantised fp64 x W^T is printed (the pages give no bound: parity unpinned)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wls
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import online_hadamard_b200 as m
+    m.load_library()
+    return m
+
+
+CASES = [wls.TINY, wls.QWEN_UP_DECODE.with_m(1), wls.QWEN_UP_DECODE.with_m(16), wls.LLAMA_UP,
+         wls.QWEN_DOWN, wls.stack_layer(0, "q", 32), wls.stack_layer(63, "down", 512),
+         wls.stack_layer(17, "k", 4)]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: f"{w.name}_M{w.M}")
+def test_linear_end_to_end(mq, wl):
+    x = wls.make_x(wl)
+    W = wls.make_w(wl)
+    s = wls.make_s(wl, W)
+    Wq, Ws, am = mq.macaq_fold_weights(W.cuda(), s.cuda())
+    y = mq.macaq_w4a4_linear(x.cuda(), am, Wq, Ws, wl.N)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(100 + wl.config)
+    rows = np.arange(wl.M) if wl.M <= 64 else np.sort(rng.choice(wl.M, 16, replace=False))
+    xf = x.float().numpy()
+    Wf = W.numpy()
+    rWq, rWs, ra = oracle.fold_weights(Wf, s.numpy())
+    rAq, rAs = oracle.act_transform_quant(xf[rows], ra)
+    ref = oracle.mx_gemm(rAq, rAs, rWq, rWs)
+    got = gu.to_np(y.float())[rows]
+    err = gu.rel_fro(got, gu.bf16_round(ref))
+    exact = xf[rows].astype(np.float64) @ Wf.astype(np.float64).T
+    q_err = gu.rel_fro(got, exact)
+    print(f"{wl.name} M={wl.M}: vs oracle {err:.2e}; W4A4 error vs fp64 x W^T {q_err:.4f} (reported)")
+    assert err <= 1e-3
+
+
+def test_linear_zero_input_gives_zero(mq):
+    M, K, N = 5, 256, 384
+    W = torch.randn(N, K, device="cuda") * 0.02
+    s = torch.rand(K, device="cuda") + 0.5
+    Wq, Ws, am = mq.macaq_fold_weights(W, s)
+    y = mq.macaq_w4a4_linear(torch.zeros(M, K, dtype=torch.bfloat16, device="cuda"), am, Wq, Ws, N)
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_linear_workspace_and_errors(mq):
+    M, K, N = 3, 64, 40
+    W = torch.randn(N, K, device="cuda")
+    s = torch.ones(K, device="cuda")
+    Wq, Ws, am = mq.macaq_fold_weights(W, s)
+    x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
+    small = torch.empty(mq.linear_workspace_bytes(M, K) - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(mq.MacaqError) as ei:
+        mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=small)
+    assert ei.value.status == -6
+    ws = torch.full((mq.linear_workspace_bytes(M, K),), 0xFF, dtype=torch.uint8, device="cuda")
+    y1 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=ws)
+    y2 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N)
+    assert torch.equal(y1, y2)
+    assert mq.macaq_device_status() == 0
