@@ -44,8 +44,9 @@
  *   - The calls validate, enqueue kernels on `stream` and return; the return value is the
  *     validation/launch status.  Errors of the asynchronous work surface at the next
  *     synchronisation; a device-side wait that gives up (it never should) sets a flag
- *     that macaq_device_status() reports.  No call allocates device memory, except as
- *     stated for macaq_fold_weights (none) -- scratch is passed in by the caller.
+ *     that macaq_device_status() reports.  No call allocates device memory: scratch is
+ *     passed in by the caller, or, for macaq_w4a4_linear_noalloc, held in a static array
+ *     of the library.
  *   - Non-finite activations or weights are out of scope (codes are then unspecified).
  */
 #ifndef MACAQ_H_
@@ -65,7 +66,8 @@ typedef enum {
     MACAQ_EALIGN = -3,     /* a pointer is not 16-byte aligned */
     MACAQ_ECUDA = -4,      /* a CUDA runtime call or kernel launch failed */
     MACAQ_ETIMEOUT = -5,   /* a bounded device-side wait gave up (see macaq_device_status) */
-    MACAQ_EWORKSPACE = -6  /* workspace smaller than the call needs */
+    MACAQ_EWORKSPACE = -6, /* workspace smaller than the call needs */
+    MACAQ_ETOOLARGE = -7   /* problem needs more than the no-allocation scratch (below) */
 } macaq_status;
 
 /* Human-readable name of a status code (static storage). */
@@ -138,6 +140,33 @@ int macaq_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, 
 int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
                      const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32,
                      void* stream);
+
+/*
+ * macaq_w4a4_linear_noalloc -- macaq_w4a4_linear for callers that cannot allocate device
+ * memory.  The paper has no counterpart: it is a deployment variant of the call above.
+ *
+ * cudaMalloc synchronises the device and can fail or fragment memory at run time, so a
+ * latency-critical serving loop that plans all of its memory up front must not call it, a
+ * plugin whose host application owns every device allocation has no allocator to call,
+ * and a plain C caller handed only device pointers for its inputs and outputs cannot
+ * obtain a buffer.  This call therefore allocates nothing: the activation codes and scales
+ * go to a static device array of MACAQ_NOALLOC_SCRATCH_BYTES inside the library, present
+ * on every GPU that loads the library until the process exits.
+ *   Arguments, layouts and results are those of macaq_w4a4_linear (without workspace).
+ *   MACAQ_ETOOLARGE (nothing launched) when macaq_linear_workspace_bytes(M, K) exceeds
+ *   MACAQ_NOALLOC_SCRATCH_BYTES.
+ *   All calls share the one array and it keeps the previous call's contents; each call
+ *   writes everything it later reads, so nothing needs clearing, but calls whose work
+ *   overlaps on the GPU (unordered streams, concurrent host threads) race on it and
+ *   corrupt each other's results -- order them on one stream.
+ *   The first call on a device looks up the array's device address once
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   CUDA stream capture begins.
+ */
+#define MACAQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int macaq_w4a4_linear_noalloc(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
+                              const uint8_t* Wq, const uint8_t* Ws, int64_t N, uint16_t* y,
+                              void* stream);
 
 /* Sticky device-side status of the current device: MACAQ_OK, or MACAQ_ETIMEOUT once a
  * bounded wait inside a kernel gave up.  Synchronises the device.  `clear` != 0 resets it. */

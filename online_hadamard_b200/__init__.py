@@ -24,7 +24,7 @@ from . import build as _build_mod
 __all__ = [
     "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
-    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status", "status_str",
+    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_w4a4_linear_noalloc", "macaq_device_status", "status_str",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -32,7 +32,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "macaq_status_str", "macaq_scale_bytes", "macaq_scale_offset", "macaq_linear_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
-    "macaq_act_quant_plain", "macaq_mxfp4_gemm", "macaq_device_status",
+    "macaq_act_quant_plain", "macaq_mxfp4_gemm", "macaq_device_status", "macaq_w4a4_linear_noalloc",
 )
 
 MACAQ_OK = 0
@@ -72,8 +72,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p]
         lib.macaq_w4a4_linear.argtypes = [p, i64, i64, p, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
+        lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
         for name in ("macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
-                     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status"):
+                     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status",
+                     "macaq_w4a4_linear_noalloc"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -192,6 +194,27 @@ def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor,
     _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
                                             _ptr(workspace), workspace.numel(), _stream(stream)),
            "macaq_w4a4_linear")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20  # MACAQ_NOALLOC_SCRATCH_BYTES of include/macaq.h
+
+
+def macaq_w4a4_linear_noalloc(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor,
+                              N: int, y=None, stream=None):
+    """macaq_w4a4_linear without a workspace: for callers that cannot allocate device memory,
+    the library keeps the activation scratch in its own static 32 MiB device array (see
+    include/macaq.h for the limit and the ordering rule).  Only y is allocated here, and
+    only when the caller does not pass it."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(act_mult, "act_mult", torch.float32, (K,))
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(Ws, "Ws", torch.uint8)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    _check(load_library().macaq_w4a4_linear_noalloc(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+                                                    _stream(stream)), "macaq_w4a4_linear_noalloc")
     return y
 
 

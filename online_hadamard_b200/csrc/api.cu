@@ -31,6 +31,8 @@ extern "C" const char* macaq_status_str(int status) {
         case MACAQ_ECUDA: return "MACAQ_ECUDA: CUDA runtime or launch failure";
         case MACAQ_ETIMEOUT: return "MACAQ_ETIMEOUT: a bounded device-side wait gave up";
         case MACAQ_EWORKSPACE: return "MACAQ_EWORKSPACE: workspace too small";
+        case MACAQ_ETOOLARGE:
+            return "MACAQ_ETOOLARGE: problem needs more scratch than the no-allocation entry point holds";
         default: return "MACAQ: unknown status";
     }
 }

@@ -3,3 +3,4 @@
 #include "api.cu"
 #include "quant.cu"
 #include "gemm.cu"
+#include "noalloc.cu"
