@@ -18,10 +18,13 @@
 //   warp 1     allocates tensor memory; one lane issues, per stage, tcgen05.cp of the
 //              scale atoms into TMEM and four tcgen05.mma (K = 64 each), then commits the
 //              stage back to the producer and, per tile, the accumulator to the epilogue.
-//   warps 2-5  epilogue: tcgen05.ld of the fp32 accumulator (warp w reads TMEM lanes of
-//              sub-partition w % 4), conversion, and stores of y.
-//   Accumulators are double-buffered in TMEM when BN <= 128 so the epilogue of one tile
-//   overlaps the mainloop of the next.  All waits are bounded (see sm100.cuh).
+//   warps 2-9  epilogue: two warps per TMEM sub-partition (warp w reads lanes of
+//              sub-partition w % 4, one half of the tile's columns each) copy the fp32
+//              accumulator into registers, hand the TMEM back to the MMA warp at once, then
+//              convert and store y, so the next tile's mainloop overlaps the stores.
+//   Scale factors are double-buffered in TMEM (alternating per k-tile), so the copy for
+//   k-tile t+1 never writes columns the MMAs of k-tile t still read.  Accumulators are
+//   double-buffered too when BN <= 128.  All waits are bounded (see sm100.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -40,7 +43,8 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
 constexpr int kStageKBytes = 128;  // code bytes per row per stage
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kEpiThreads = 256;
 
 template <int BN>
 struct TileCfg {
@@ -52,10 +56,10 @@ struct TileCfg {
     static constexpr int kStageBytes = kPBytes + kQBytes + kSFPBytes + kSFQBytes;
     static constexpr int kNumAcc = BN <= 128 ? 2 : 1;
     static constexpr int kAccStride = ((BN + 31) / 32) * 32;
-    static constexpr int kSFPCol = kNumAcc * kAccStride;           // 2 groups x 4 columns
-    static constexpr int kSFQCol = kSFPCol + 8;
     static constexpr int kSFQColsPerGroup = 4 * kQBlocks;
-    static constexpr int kColsUsed = kSFQCol + 2 * kSFQColsPerGroup;
+    static constexpr int kSFBufCols = 8 + 2 * kSFQColsPerGroup;    // P: 2 groups x 4, then Q
+    static constexpr int kSFBase = kNumAcc * kAccStride;           // two scale buffers follow
+    static constexpr int kColsUsed = kSFBase + 2 * kSFBufCols;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                    : kColsUsed <= 256 ? 256 : 512;
     static_assert(kColsUsed <= 512, "tensor memory budget");
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 128);
+            mbar_init(&acc_empty[a], kEpiThreads);
         }
         fence_mbar_init();
         prefetch_tmap(&tmap_p);
@@ -206,6 +210,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
+            uint32_t sfbuf = 0;
             for (int tile = blockIdx.x; tile < num_tiles && !abort; tile += gridDim.x) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort)) break;
                 tc_fence_after();
@@ -217,20 +222,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t sq = sp + Cfg::kPBytes;
                     const uint32_t ssfp = sq + Cfg::kQBytes;
                     const uint32_t ssfq = ssfp + Cfg::kSFPBytes;
+                    const uint32_t tsfp = tmem_base + Cfg::kSFBase + sfbuf * Cfg::kSFBufCols;
+                    const uint32_t tsfq = tsfp + 8;
+                    sfbuf ^= 1u;
 #pragma unroll
                     for (int g = 0; g < 2; ++g) {
-                        tc_cp_sf(tmem_base + Cfg::kSFPCol + 4 * g, desc_sf(ssfp + 512 * g));
+                        tc_cp_sf(tsfp + 4 * g, desc_sf(ssfp + 512 * g));
 #pragma unroll
                         for (int i = 0; i < Cfg::kQBlocks; ++i)
-                            tc_cp_sf(tmem_base + Cfg::kSFQCol + Cfg::kSFQColsPerGroup * g + 4 * i,
-                                     desc_sf(ssfq + 1024 * i + 512 * g));
+                            tc_cp_sf(tsfq + Cfg::kSFQColsPerGroup * g + 4 * i, desc_sf(ssfq + 1024 * i + 512 * g));
                     }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t g = j >> 1;
                         const uint32_t id = (j & 1) * 2;  // byte of the scale word: blocks 2j%4, 2j%4+1
-                        const uint32_t sfa = (tmem_base + Cfg::kSFPCol + 4 * g) | (id << 30);
-                        const uint32_t sfb = (tmem_base + Cfg::kSFQCol + Cfg::kSFQColsPerGroup * g) | (id << 30);
+                        const uint32_t sfa = (tsfp + 4 * g) | (id << 30);
+                        const uint32_t sfb = (tsfq + Cfg::kSFQColsPerGroup * g) | (id << 30);
                         tc_mma_mxf4(d_tmem, desc_sw128(sp + 32 * j), desc_sw128(sq + 32 * j),
                                     idesc | (id << 29) | (id << 4), sfa, sfb, (kt | j) != 0 ? 1u : 0u);
                     }
@@ -250,7 +257,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int sub = warp & 3;  // TMEM sub-partition this warp may read
+        constexpr int kHalf = BN / 2;            // columns per epilogue warp
+        constexpr int kChunk = kHalf >= 32 ? 32 : kHalf;
+        const int sub = warp & 3;                // TMEM sub-partition this warp may read
+        const int half = (warp - 2) >> 2;        // which half of the tile's columns
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < num_tiles && !abort; tile += gridDim.x) {
@@ -259,30 +269,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (!mbar_wait(&acc_full[acc], acc_phase, &abort)) break;
             tc_fence_after();
             const int64_t prow = static_cast<int64_t>(pt) * kBM + sub * 32 + lane;
-            const uint32_t tbase = tmem_base + acc * Cfg::kAccStride + (static_cast<uint32_t>(sub * 32) << 16);
-            if constexpr (BN % 32 == 0) {
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + c, r);
-                    tmem_ld_wait();
-                    store_chunk<32, SWAP>(prm, prow, static_cast<int64_t>(qt) * BN + c, r);
-                }
-            } else {
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(tbase + c, r);
-                    tmem_ld_wait();
-                    store_chunk<16, SWAP>(prm, prow, static_cast<int64_t>(qt) * BN + c, r);
-                }
-            }
+            const uint32_t tbase = tmem_base + acc * Cfg::kAccStride + half * kHalf +
+                                   (static_cast<uint32_t>(sub * 32) << 16);
+            uint32_t v[kHalf];
+#pragma unroll
+            for (int c = 0; c < kHalf; c += kChunk) tmem_ld_cols<kChunk>(tbase + c, v + c);
+            tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
+            mbar_arrive(&acc_empty[acc]);  // accumulator is in registers: TMEM is free again
             if (++acc == Cfg::kNumAcc) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
+            const int64_t q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
+#pragma unroll
+            for (int c = 0; c < kHalf; c += kChunk) store_chunk<kChunk, SWAP>(prm, prow, q0 + c, v + c);
         }
     }
 

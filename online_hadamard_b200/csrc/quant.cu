@@ -1,7 +1,7 @@
 // quant.cu -- MXFP4 quantisation kernels along K, with the online MACaQ transform.
 //
-//   act_transform: u = fl32(x * act_mult), block-Hadamard b = 32 (FWHT in registers and
-//                  warp shuffles), E8M0 scale, E2M1 RTN codes       (activations, online)
+//   act_transform: u = fl32(x * act_mult), block-Hadamard b = 32 (FWHT in registers),
+//                  E8M0 scale, E2M1 RTN codes                       (activations, online)
 //   weight_fold:   u = fl32(W * fl32(s * c)), same transform and quantisation (weights,
 //                  offline; also writes act_mult = fl32(c / s))
 //   plain:         MXFP4 of x with no scale and no transform       (baseline)
@@ -10,14 +10,15 @@
 // Activations", Abstract: per-channel scale + block-Hadamard online on the activations,
 // inverse transforms absorbed into the weights, MXFP4 W4A4, round-to-nearest weights.
 //
-// Work split: one warp task = one row x 256 consecutive elements (8 blocks of 32).  Lane
-// quad q (lanes 4q..4q+3) owns block 8*task+q; each lane owns 8 consecutive elements,
-// loaded as one 16-byte vector (bf16) or two (fp32).  Butterfly stages h = 1, 2, 4 stay
-// in a lane's registers; h = 8, 16 cross lanes with __shfl_xor (masks 1, 2).  Every fp32
-// operation is an explicit round-to-nearest intrinsic, so the compiler cannot contract
-// the scale into the first butterfly, and the result is bit-identical to the canonical
-// sequential order.  The kernel is HBM-bound: 2 (or 4) bytes in, 0.53 bytes out per
-// element.
+// Work split: one thread owns one 32-element block column and walks a group of rows, so
+// its 32 multipliers stay in registers and the whole 32-point butterfly runs in its
+// registers with no cross-lane traffic.  A warp covers 32 consecutive blocks (2 KB of
+// bf16) of one row: its four 16-byte loads per row touch every sector of that span, and
+// its 16-byte code stores are contiguous.  Two rows are loaded before either is used to
+// keep enough bytes in flight.  Every fp32 operation is an explicit round-to-nearest
+// intrinsic (scalar or the sm_100 packed f32x2 form), so the scale cannot be contracted
+// into the first butterfly and the result is bit-identical to the canonical sequential
+// order.  The kernel is HBM-bound: 2 (or 4) bytes in, 0.53 bytes out per element.
 #include <cstdint>
 #include <cmath>
 #include <vector>
@@ -29,12 +30,12 @@ namespace macaq {
 
 enum class QuantMode { kActTransform = 0, kWeightFold = 1, kPlain = 2 };
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;
+constexpr int kQuantThreads = 128;
 
-// Eight E2M1 codes (magnitudes only) of |q0..q7| packed two per byte, element 2j in the
-// low nibble: cvt.rn.satfinite.e2m1x2 puts its first source in the high nibble.
-__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&q)[8]) {
+// Eight E2M1 codes of q0..q7 (non-negative) packed two per byte, element 2j in the low
+// nibble: cvt.rn.satfinite.e2m1x2 puts its first source in the high nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float q0, float q1, float q2, float q3, float q4, float q5,
+                                               float q6, float q7) {
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -43,181 +44,201 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&q)[8]) {
         "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
-        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+        : "f"(q0), "f"(q1), "f"(q2), "f"(q3), "f"(q4), "f"(q5), "f"(q6), "f"(q7));
     return out;
 }
 
+// Sign bits of eight values placed on the sign bit (bit 3) of their nibbles.
+__device__ __forceinline__ uint32_t sign_nibbles(const float2* v) {
+    uint32_t s = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        s |= (__float_as_uint(v[j].x) >> 31) << (8 * j + 3);
+        s |= (__float_as_uint(v[j].y) >> 31) << (8 * j + 7);
+    }
+    return s;
+}
+
+// 32 raw inputs of one block as 16 pairs (bf16 widened exactly, or fp32).
 template <QuantMode MODE>
-struct QuantLoad {
-    float x[8];
-    float m[8];
+struct RawBlock {
+    uint4 w[MODE == QuantMode::kWeightFold ? 8 : 4];
 };
 
 template <QuantMode MODE>
-__device__ __forceinline__ void load_item(const void* __restrict__ in, const float* __restrict__ mult,
-                                          const float* __restrict__ s, double c, int64_t row_off,
-                                          int64_t k0, QuantLoad<MODE>& it) {
+__device__ __forceinline__ void load_block(const void* __restrict__ in, int64_t off, RawBlock<MODE>& b) {
     if constexpr (MODE == QuantMode::kWeightFold) {
-        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(in) + row_off + k0);
-        const float4 a = __ldcs(p);
-        const float4 b = __ldcs(p + 1);
-        it.x[0] = a.x; it.x[1] = a.y; it.x[2] = a.z; it.x[3] = a.w;
-        it.x[4] = b.x; it.x[5] = b.y; it.x[6] = b.z; it.x[7] = b.w;
-        const float4* sp = reinterpret_cast<const float4*>(s + k0);
-        const float4 s0 = __ldg(sp);
-        const float4 s1 = __ldg(sp + 1);
-        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(in) + off);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) it.m[j] = __double2float_rn(__dmul_rn(static_cast<double>(sv[j]), c));
+        for (int j = 0; j < 8; ++j) b.w[j] = __ldcs(p + j);
     } else {
-        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in) + row_off + k0));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(in) + off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b.w[j] = __ldcs(p + j);
+    }
+}
+
+template <QuantMode MODE>
+__device__ __forceinline__ void widen(const RawBlock<MODE>& b, float2 (&u)[16]) {
+    if constexpr (MODE == QuantMode::kWeightFold) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            u[2 * j] = make_float2(__uint_as_float(b.w[j].x), __uint_as_float(b.w[j].y));
+            u[2 * j + 1] = make_float2(__uint_as_float(b.w[j].z), __uint_as_float(b.w[j].w));
+        }
+    } else {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            it.x[2 * j] = __uint_as_float(w[j] << 16);            // bf16 -> fp32 is exact
-            it.x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
-        if constexpr (MODE == QuantMode::kActTransform) {
-            const float4* mp = reinterpret_cast<const float4*>(mult + k0);
-            const float4 m0 = __ldg(mp);
-            const float4 m1 = __ldg(mp + 1);
-            it.m[0] = m0.x; it.m[1] = m0.y; it.m[2] = m0.z; it.m[3] = m0.w;
-            it.m[4] = m1.x; it.m[5] = m1.y; it.m[6] = m1.z; it.m[7] = m1.w;
+            const uint32_t w[4] = {b.w[j].x, b.w[j].y, b.w[j].z, b.w[j].w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t)  // bf16 -> fp32 is exact: the bits move up 16 places
+                u[4 * j + t] = make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u));
         }
     }
 }
 
-// Scale + FWHT-32 of the block held by a lane quad; `sub` = lane % 4 = element bits 3-4.
-template <QuantMode MODE>
-__device__ __forceinline__ void transform(QuantLoad<MODE>& it, int sub) {
-    if constexpr (MODE == QuantMode::kPlain) return;
-    float (&u)[8] = it.x;
+// Scale by the per-channel multiplier and apply the unnormalised 32-point Walsh-Hadamard
+// butterfly in the canonical stage order h = 1, 2, 4, 8, 16.  u[p] holds elements 2p, 2p+1.
+__device__ __forceinline__ void scale_fwht32(float2 (&u)[16], const float2 (&m)[16]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[j] = __fmul_rn(u[j], it.m[j]);
+    for (int p = 0; p < 16; ++p) u[p] = __fmul2_rn(u[p], m[p]);
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
+    for (int p = 0; p < 16; ++p) {  // h = 1: the two halves of a pair
+        const float a = u[p].x, b = u[p].y;
+        u[p] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if ((j & h) == 0) {
-                const float a = u[j], b = u[j + h];
-                u[j] = __fadd_rn(a, b);
-                u[j + h] = __fsub_rn(a, b);
+    for (int hp = 1; hp < 16; hp <<= 1) {  // h = 2 hp: whole pairs, packed
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            if ((p & hp) == 0) {
+                const float2 a = u[p], b = u[p + hp];
+                u[p] = __fadd2_rn(a, b);
+                u[p + hp] = __fadd2_rn(a, make_float2(-b.x, -b.y));  // a - b, exactly one rounding
             }
         }
     }
-#pragma unroll
-    for (int s = 1; s <= 2; s <<= 1) {  // h = 8 (lane bit 0), h = 16 (lane bit 1)
-        const bool upper = (sub & s) != 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float p = __shfl_xor_sync(0xFFFFFFFFu, u[j], s);
-            // lower partner holds u_i and keeps u_i + u_{i+h}; upper holds u_{i+h}, keeps u_i - u_{i+h}
-            u[j] = upper ? __fsub_rn(p, u[j]) : __fadd_rn(u[j], p);
-        }
-    }
 }
 
-// E8M0 scale and packed codes of the block; returns the scale byte, writes 4 code bytes.
-__device__ __forceinline__ uint32_t quantize_block(const float (&v)[8], uint32_t& packed) {
+// E8M0 scale byte and the 16 code bytes of one transformed block.
+__device__ __forceinline__ uint32_t quantize32(const float2 (&v)[16], uint4& codes) {
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    for (int p = 0; p < 16; ++p) amax = fmaxf(amax, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
     const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
     const uint32_t e = E >= 3u ? E - 2u : 0u;
-    const float inv_scale = __uint_as_float((254u - e) << 23);  // 2^(127 - e), a normal float
-    float q[8];
-    uint32_t signs = 0;
+    const float inv = __uint_as_float((254u - e) << 23);  // 2^(127 - e), a normal float
+    uint32_t w[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        q[j] = __fmul_rn(fabsf(v[j]), inv_scale);  // exact unless far below the E2M1 grid
-        signs |= (__float_as_uint(v[j]) >> 31) << (4 * j + 3);
+    for (int j = 0; j < 4; ++j) {
+        const float2* q = v + 4 * j;
+        w[j] = cvt_e2m1x8(__fmul_rn(fabsf(q[0].x), inv), __fmul_rn(fabsf(q[0].y), inv),
+                          __fmul_rn(fabsf(q[1].x), inv), __fmul_rn(fabsf(q[1].y), inv),
+                          __fmul_rn(fabsf(q[2].x), inv), __fmul_rn(fabsf(q[2].y), inv),
+                          __fmul_rn(fabsf(q[3].x), inv), __fmul_rn(fabsf(q[3].y), inv)) |
+               sign_nibbles(q);
     }
-    packed = cvt_e2m1x8(q) | signs;
+    codes = make_uint4(w[0], w[1], w[2], w[3]);
     return e;
 }
 
 template <QuantMode MODE>
+__device__ __forceinline__ void process_block(const RawBlock<MODE>& raw, const float2 (&m)[16], uint8_t* codes_row,
+                                              uint8_t* scale_byte) {
+    float2 u[16];
+    widen<MODE>(raw, u);
+    if constexpr (MODE != QuantMode::kPlain) scale_fwht32(u, m);
+    uint4 c;
+    const uint32_t e = quantize32(u, c);
+    *reinterpret_cast<uint4*>(codes_row) = c;
+    *scale_byte = static_cast<uint8_t>(e);
+}
+
+// One thread = (group of `rpg` rows) x (one 32-block column), columns fastest; threads of
+// padded block columns (kb >= K/32) write the zero scale bytes of their rows.
+template <QuantMode MODE>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
-    const void* __restrict__ in, int64_t R, int64_t K, const float* __restrict__ mult,
-    const float* __restrict__ s, double c, float* __restrict__ act_mult_out,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const void* __restrict__ in, int64_t R, int64_t K, int64_t rpg, const float* __restrict__ mult,
+    const float* __restrict__ s, double c, float* __restrict__ act_mult_out, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
     griddep_launch_dependents();
-    const int lane = threadIdx.x & 31;
-    const int quad = lane >> 2;
-    const int sub = lane & 3;
     const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
-    const int64_t groups = kbp / 8;  // warp tasks per row
-    const int64_t tasks = R * groups;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kQuantThreads / 32);
-    const int64_t w0 = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
-
-    for (int64_t base = w0; base < tasks; base += warps * kQuantUnroll) {
-        QuantLoad<MODE> it[kQuantUnroll];
-        bool real[kQuantUnroll];
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+    const int64_t kb = item % kbp;
+    const int64_t r0 = (item / kbp) * rpg;
+    if (r0 >= R) return;
+    const int64_t r1 = r0 + rpg < R ? r0 + rpg : R;
+    if (kb >= kb_real) {
+        for (int64_t r = r0; r < r1; ++r) scales[scale_offset(r, kb, kbp)] = 0;
+        return;
+    }
+    const int64_t k0 = kb * 32;
+    float2 m[16];
+    if constexpr (MODE == QuantMode::kActTransform) {
+        const float4* mp = reinterpret_cast<const float4*>(mult + k0);
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t t = base + u * warps;
-            const int64_t r = t / groups;
-            const int64_t kb = (t - r * groups) * 8 + quad;
-            real[u] = t < tasks && kb < kb_real;
-            if (real[u]) load_item<MODE>(in, mult, s, c, r * K, kb * 32 + sub * 8, it[u]);
+        for (int j = 0; j < 8; ++j) {
+            const float4 t = __ldg(mp + j);
+            m[2 * j] = make_float2(t.x, t.y);
+            m[2 * j + 1] = make_float2(t.z, t.w);
         }
+    } else if constexpr (MODE == QuantMode::kWeightFold) {
+        const bool first = r0 == 0;
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t t = base + u * warps;
-            if (t >= tasks) break;  // warp-uniform
-            const int64_t r = t / groups;
-            const int64_t kb = (t - r * groups) * 8 + quad;
-            if (!real[u]) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) it[u].x[j] = 0.0f;
-            }
-            transform<MODE>(it[u], sub);
-            uint32_t packed;
-            const uint32_t e = quantize_block(it[u].x, packed);
-            if (real[u]) {
-                *reinterpret_cast<uint32_t*>(codes + r * (K / 2) + kb * 16 + sub * 4) = packed;
-                if (sub == 0) scales[scale_offset(r, kb, kbp)] = static_cast<uint8_t>(e);
-                if constexpr (MODE == QuantMode::kWeightFold) {
-                    if (r == 0) {
-                        const int64_t k0 = kb * 32 + sub * 8;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            act_mult_out[k0 + j] =
-                                __double2float_rn(__ddiv_rn(c, static_cast<double>(s[k0 + j])));
-                    }
-                }
-            } else if (sub == 0) {
-                scales[scale_offset(r, kb, kbp)] = 0;  // padded block of a real row
+        for (int p = 0; p < 16; ++p) {
+            const double s0 = static_cast<double>(s[k0 + 2 * p]);
+            const double s1 = static_cast<double>(s[k0 + 2 * p + 1]);
+            m[p] = make_float2(__double2float_rn(__dmul_rn(s0, c)), __double2float_rn(__dmul_rn(s1, c)));
+            if (first) {
+                act_mult_out[k0 + 2 * p] = __double2float_rn(__ddiv_rn(c, s0));
+                act_mult_out[k0 + 2 * p + 1] = __double2float_rn(__ddiv_rn(c, s1));
             }
         }
     }
+    int64_t r = r0;
+    for (; r + 1 < r1; r += 2) {
+        RawBlock<MODE> b0, b1;
+        load_block<MODE>(in, r * K + k0, b0);
+        load_block<MODE>(in, (r + 1) * K + k0, b1);
+        process_block<MODE>(b0, m, codes + r * (K / 2) + kb * 16, scales + scale_offset(r, kb, kbp));
+        process_block<MODE>(b1, m, codes + (r + 1) * (K / 2) + kb * 16, scales + scale_offset(r + 1, kb, kbp));
+    }
+    if (r < r1) {
+        RawBlock<MODE> b0;
+        load_block<MODE>(in, r * K + k0, b0);
+        process_block<MODE>(b0, m, codes + r * (K / 2) + kb * 16, scales + scale_offset(r, kb, kbp));
+    }
 }
 
-int quant_grid(int64_t R, int64_t K) {
-    const int64_t tasks = R * (padded_blocks(K) / 8);
-    const int64_t per_block = (kQuantThreads / 32) * kQuantUnroll;
-    int64_t blocks = (tasks + per_block - 1) / per_block;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
-    if (blocks > cap) blocks = cap;
-    return static_cast<int>(blocks < 1 ? 1 : blocks);
+// Rows per thread: enough threads to fill the GPU, rows walked by each otherwise.
+static int64_t quant_rows_per_thread(int64_t R, int64_t K) {
+    const int64_t cols = padded_blocks(K);
+    const int64_t target = static_cast<int64_t>(sm_count()) * 16 * 32;
+    int64_t rpg = (R * cols + target - 1) / target;
+    if (rpg < 1) rpg = 1;
+    return rpg;
+}
+
+static unsigned quant_blocks(int64_t R, int64_t K, int64_t rpg) {
+    const int64_t items = padded_blocks(K) * ((R + rpg - 1) / rpg);
+    return static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
 }
 
 // Launch helpers used by the C entry points and by the fused linear.
 int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
                                uint8_t* Aq, uint8_t* As, cudaStream_t stream) {
-    mx_quant_kernel<QuantMode::kActTransform><<<quant_grid(M, K), kQuantThreads, 0, stream>>>(
-        x, M, K, act_mult, nullptr, 0.0, nullptr, Aq, As);
+    const int64_t rpg = quant_rows_per_thread(M, K);
+    mx_quant_kernel<QuantMode::kActTransform><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
+        x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As);
     return launch_status();
 }
 
 int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                            cudaStream_t stream) {
-    mx_quant_kernel<QuantMode::kPlain><<<quant_grid(M, K), kQuantThreads, 0, stream>>>(
-        x, M, K, nullptr, nullptr, 0.0, nullptr, Aq, As);
+    const int64_t rpg = quant_rows_per_thread(M, K);
+    mx_quant_kernel<QuantMode::kPlain><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
+        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As);
     return launch_status();
 }
 
@@ -257,7 +278,8 @@ extern "C" int macaq_fold_weights(const float* W, int64_t N, int64_t K, const fl
     for (float v : hs)
         if (!(v > 0.0f) || !std::isfinite(v)) return MACAQ_EINVAL;
     const double c = 1.0 / std::sqrt(32.0);  // correctly rounded (IEEE sqrt and divide)
-    mx_quant_kernel<QuantMode::kWeightFold><<<quant_grid(N, K), kQuantThreads, 0, st>>>(
-        W, N, K, nullptr, s, c, act_mult, Wq, Ws);
+    const int64_t rpg = quant_rows_per_thread(N, K);
+    mx_quant_kernel<QuantMode::kWeightFold><<<quant_blocks(N, K, rpg), kQuantThreads, 0, st>>>(
+        W, N, K, rpg, nullptr, s, c, act_mult, Wq, Ws);
     return launch_status();
 }
