@@ -145,11 +145,12 @@ class Layer:
         W = wls.make_w(wl)
         s = wls.make_s(wl, W)
         x = wls.make_x(wl)
-        footprint = (wl.M * wl.K * 2 + wl.N * wl.K * 0.53125 + wl.M * wl.N * 2 + mq.linear_workspace_bytes(wl.M, wl.K))
+        footprint = wl.M * wl.K * 2 + wl.N * wl.K * 0.53125 + wl.M * wl.N * 2 + wl.M * wl.K * 0.53125
         self.copies = copies or max(2, math.ceil(3 * L2_BYTES / footprint))
         Wd = W.to(device)
         sd = s.to(device)
         self.Wq, self.Ws, self.am, self.x, self.y, self.ws, self.Aq, self.As = [], [], [], [], [], [], [], []
+        self.gws = []
         torch.cuda.synchronize(device)
         t0 = time.perf_counter()
         for _ in range(self.copies):
@@ -164,7 +165,9 @@ class Layer:
         for _ in range(self.copies):
             self.x.append(xd.clone())
             self.y.append(torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=device))
-            self.ws.append(torch.empty(mq.linear_workspace_bytes(wl.M, wl.K), dtype=torch.uint8, device=device))
+            self.ws.append(torch.empty(mq.linear_workspace_bytes(wl.M, wl.N, wl.K), dtype=torch.uint8, device=device))
+            self.gws.append(torch.empty(max(mq.gemm_workspace_bytes(wl.M, wl.N, wl.K), 1), dtype=torch.uint8,
+                                        device=device))
             Aq, As = mq.macaq_act_transform_quant(xd, self.am[0])
             self.Aq.append(Aq)
             self.As.append(As)
@@ -180,13 +183,13 @@ class Layer:
     def gemm(self, i):
         c = i % self.copies
         self.mq.macaq_mxfp4_gemm(self.Aq[c], self.As[c], self.Wq[c], self.Ws[c], self.wl.M, self.wl.N, self.wl.K,
-                                 y=self.y[c])
+                                 y=self.y[c], workspace=self.gws[c])
 
     def plain(self, i):
         c = i % self.copies
         self.mq.macaq_act_quant_plain(self.x[c], Aq=self.Aq[c], As=self.As[c])
         self.mq.macaq_mxfp4_gemm(self.Aq[c], self.As[c], self.Wq[c], self.Ws[c], self.wl.M, self.wl.N, self.wl.K,
-                                 y=self.y[c])
+                                 y=self.y[c], workspace=self.gws[c])
 
     def transform_only(self, i):
         c = i % self.copies
@@ -200,7 +203,40 @@ class Layer:
         self.y_host.copy_(self.y[c], non_blocking=True)
 
 
-def time_loop(fn, steps, warmup, device):
+class GraphLoop:
+    """`steps` calls of fn(i) captured once into a CUDA graph, replayed as one launch, so the
+    timed region holds only GPU work (no per-call host launch overhead)."""
+
+    def __init__(self, fn, steps, warmup, device, offset=0):
+        self.device = device
+        for i in range(warmup):
+            fn(offset + i)
+        torch.cuda.synchronize(device)
+        self.stream = torch.cuda.Stream(device)
+        self.graph = torch.cuda.CUDAGraph()
+        self.stream.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(self.stream):
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                for i in range(steps):
+                    fn(offset + warmup + i)
+        torch.cuda.current_stream(device).wait_stream(self.stream)
+        torch.cuda.synchronize(device)
+        self.graph.replay()  # one untimed replay
+        torch.cuda.synchronize(device)
+
+    def time_ms(self):
+        """Total time of one replay, by CUDA events on the replaying stream."""
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        self.graph.replay()
+        e1.record()
+        torch.cuda.synchronize(self.device)
+        return e0.elapsed_time(e1)
+
+
+def time_eager(fn, steps, warmup, device):
+    """ms per call of fn launched eagerly from Python (host launch overhead included)."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize(device)
@@ -211,7 +247,15 @@ def time_loop(fn, steps, warmup, device):
         fn(warmup + i)
     e1.record()
     torch.cuda.synchronize(device)
-    return e0.elapsed_time(e1) / steps  # ms per call
+    return e0.elapsed_time(e1) / steps
+
+
+def time_loop(fn, steps, warmup, device):
+    """ms per call of fn, from a graph-captured loop of `steps` calls."""
+    g = GraphLoop(fn, steps, warmup, device)
+    ms = g.time_ms() / steps
+    del g
+    return ms
 
 
 # --------------------------------------------------------------------------- CPU baseline
@@ -282,7 +326,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--profile", default=None, metavar="WORKLOAD",
+                    help="run each kernel of one workload three times (for ncu captures) and exit; "
+                         "WORKLOAD is a name from workloads.py, optionally with _M<m>")
     args = ap.parse_args()
+    if args.profile:
+        profile_kernels(args.profile)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
@@ -320,25 +370,20 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # ---- headline: the fused linear
-    for i in range(args.warmup):
-        layer.linear(i)
+    # ---- headline: the fused linear, K steps captured in one CUDA graph
+    loop = GraphLoop(layer.linear, args.steps, args.warmup, device)
     torch.cuda.synchronize(device)
     barrier()
     torch.cuda.synchronize(device)
     clocks = ClockSampler(local)
     clocks.start()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        layer.linear(args.warmup + i)
-    e1.record()
+    ms_total = loop.time_ms()
     torch.cuda.synchronize(device)
     barrier()
     torch.cuda.synchronize(device)
     clk = clocks.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    del loop
+    ms = max_over_ranks(ms_total / args.steps)
     value = world * wl.flops / (ms * 1e-3) / 1e12
 
     # ---- dominant kernel, the comparators and end to end (same rotation)
@@ -346,7 +391,7 @@ def main():
     ms_plain = time_loop(layer.plain, args.steps, args.warmup, device)
     ms_xform = time_loop(layer.transform_only, args.steps, args.warmup, device)
     e2e_steps = max(3, min(args.steps, 10))
-    ms_e2e = max_over_ranks(time_loop(layer.e2e, e2e_steps, 3, device))
+    ms_e2e = max_over_ranks(time_eager(layer.e2e, e2e_steps, 3, device))
     gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
     xform_bytes = wl.M * wl.K * 2 + wl.M * wl.K * (0.5 + 1 / 32) + wl.K * 4
     traffic = recorded_traffic("mxf4_gemm_128x256:" + wl.name)
@@ -387,6 +432,28 @@ def main():
         print(json.dumps(out))
     if dist is not None:
         dist.destroy_process_group()
+
+
+def profile_kernels(name):
+    """Launch sequence for ncu: fold once, then 3 x (transform+quant, plain quant, GEMM)."""
+    import online_hadamard_b200 as mq
+    base, _, m = name.partition("_M")
+    wl = next(w for w in wls.ALL if w.name == base)
+    if m:
+        wl = wl.with_m(int(m))
+    W = wls.make_w(wl)
+    s = wls.make_s(wl, W)
+    x = wls.make_x(wl).cuda()
+    Wq, Ws, am = mq.macaq_fold_weights(W.cuda(), s.cuda())
+    Aq, As = mq.macaq_act_transform_quant(x, am)
+    y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device="cuda")
+    gws = torch.empty(max(mq.gemm_workspace_bytes(wl.M, wl.N, wl.K), 1), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        mq.macaq_act_transform_quant(x, am, Aq=Aq, As=As)
+        mq.macaq_act_quant_plain(x, Aq=Aq, As=As)
+        mq.macaq_mxfp4_gemm(Aq, As, Wq, Ws, wl.M, wl.N, wl.K, y=y, workspace=gws)
+    torch.cuda.synchronize()
+    print(f"profiled {wl.name} M={wl.M} K={wl.K} N={wl.N}")
 
 
 def secondary(mq, device, peaks, args):

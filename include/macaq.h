@@ -80,9 +80,15 @@ size_t macaq_scale_bytes(int64_t rows, int64_t K);
 /* Offset of the scale byte of (row r, 32-block kb) in that buffer (-1 if out of range). */
 int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
 
-/* Bytes of scratch macaq_w4a4_linear needs for M x K activations: their MXFP4 codes
- * (M*K/2, rounded up to 256) plus scales (macaq_scale_bytes(M, K)). */
-size_t macaq_linear_workspace_bytes(int64_t M, int64_t K);
+/* Bytes of scratch macaq_mxfp4_gemm uses for its stream-K schedule on the current device
+ * (a flag and a 128-row fp32 partial-sum slot per CTA of the persistent grid; depends on M
+ * and the device's SM count). */
+size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Bytes of scratch macaq_w4a4_linear needs on the current device: the activations' MXFP4
+ * codes (M*K/2) and scales (macaq_scale_bytes(M, K)), each rounded up to 256, then
+ * macaq_gemm_workspace_bytes(M, N, K). */
+size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
  * macaq_fold_weights -- offline weight preparation (Abstract: "absorbing the corresponding
@@ -119,9 +125,9 @@ int macaq_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const flo
  *   x         in   bf16 [M][K];  act_mult in fp32 [K]
  *   Wq, Ws    in   folded weights from macaq_fold_weights (N rows)
  *   y         out  bf16 [M][N]
- *   workspace in   scratch of at least macaq_linear_workspace_bytes(M, K) bytes
- *                  (MACAQ_EWORKSPACE otherwise); its contents on return are unspecified
- *                  and calls sharing one workspace must be stream-ordered.
+ *   workspace in   scratch of at least macaq_linear_workspace_bytes(M, N, K) bytes
+ *                  (MACAQ_EWORKSPACE otherwise); its contents on entry and on return are
+ *                  unspecified and calls sharing one workspace must be stream-ordered.
  */
 int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
                       const uint8_t* Wq, const uint8_t* Ws, int64_t N, uint16_t* y,
@@ -133,13 +139,17 @@ int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_
  *
  * macaq_act_quant_plain: MXFP4 quantisation of x with no scale and no transform.
  * macaq_mxfp4_gemm: y = dec(A) dec(W)^T for already-quantised operands, fp32 accumulate;
- *   y is bf16 [M][N] (y_is_fp32 = 0) or fp32 [M][N] (y_is_fp32 = 1).
+ *   y is bf16 [M][N] (y_is_fp32 = 0) or fp32 [M][N] (y_is_fp32 = 1).  With a workspace of
+ *   macaq_gemm_workspace_bytes(M, N, K) the GEMM balances its last wave with a stream-K
+ *   split of the K steps (partial sums added in a fixed order, so results are
+ *   deterministic); with workspace = NULL it runs a data-parallel schedule.  Both
+ *   schedules accumulate in fp32 and agree within fp32 summation order.
  */
 int macaq_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                           void* stream);
 int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
                      const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32,
-                     void* stream);
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * macaq_w4a4_linear_noalloc -- macaq_w4a4_linear for callers that cannot allocate device
@@ -153,8 +163,10 @@ int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint
  * go to a static device array of MACAQ_NOALLOC_SCRATCH_BYTES inside the library, present
  * on every GPU that loads the library until the process exits.
  *   Arguments, layouts and results are those of macaq_w4a4_linear (without workspace).
- *   MACAQ_ETOOLARGE (nothing launched) when macaq_linear_workspace_bytes(M, K) exceeds
- *   MACAQ_NOALLOC_SCRATCH_BYTES.
+ *   MACAQ_ETOOLARGE (nothing launched) when the activations' codes and scales (the first
+ *   part of macaq_linear_workspace_bytes(M, N, K)) exceed MACAQ_NOALLOC_SCRATCH_BYTES; the
+ *   GEMM uses its stream-K schedule when the whole workspace fits, else its data-parallel
+ *   one.
  *   All calls share the one array and it keeps the previous call's contents; each call
  *   writes everything it later reads, so nothing needs clearing, but calls whose work
  *   overlaps on the GPU (unordered streams, concurrent host threads) race on it and

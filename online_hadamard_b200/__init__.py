@@ -22,7 +22,7 @@ import torch
 from . import build as _build_mod
 
 __all__ = [
-    "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes",
+    "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes", "gemm_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_w4a4_linear_noalloc", "macaq_device_status", "status_str",
     "EXPORTED_SYMBOLS",
@@ -31,6 +31,7 @@ __all__ = [
 # Every symbol include/macaq.h declares.
 EXPORTED_SYMBOLS = (
     "macaq_status_str", "macaq_scale_bytes", "macaq_scale_offset", "macaq_linear_workspace_bytes",
+    "macaq_gemm_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
     "macaq_act_quant_plain", "macaq_mxfp4_gemm", "macaq_device_status", "macaq_w4a4_linear_noalloc",
 )
@@ -64,12 +65,14 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_scale_bytes.restype = sz
         lib.macaq_scale_offset.argtypes = [i64, i64, i64]
         lib.macaq_scale_offset.restype = i64
-        lib.macaq_linear_workspace_bytes.argtypes = [i64, i64]
+        lib.macaq_linear_workspace_bytes.argtypes = [i64, i64, i64]
         lib.macaq_linear_workspace_bytes.restype = sz
+        lib.macaq_gemm_workspace_bytes.argtypes = [i64, i64, i64]
+        lib.macaq_gemm_workspace_bytes.restype = sz
         lib.macaq_fold_weights.argtypes = [p, i64, i64, p, p, p, p, p]
         lib.macaq_act_transform_quant.argtypes = [p, i64, i64, p, p, p, p]
         lib.macaq_act_quant_plain.argtypes = [p, i64, i64, p, p, p]
-        lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p]
+        lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p, sz, p]
         lib.macaq_w4a4_linear.argtypes = [p, i64, i64, p, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
         lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
@@ -121,8 +124,14 @@ def scale_offset(r: int, kb: int, K: int) -> int:
     return int(load_library().macaq_scale_offset(r, kb, K))
 
 
-def linear_workspace_bytes(M: int, K: int) -> int:
-    return int(load_library().macaq_linear_workspace_bytes(M, K))
+def linear_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Scratch bytes macaq_w4a4_linear needs on the current device."""
+    return int(load_library().macaq_linear_workspace_bytes(M, N, K))
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Scratch bytes of the GEMM's stream-K schedule on the current device."""
+    return int(load_library().macaq_gemm_workspace_bytes(M, N, K))
 
 
 def macaq_fold_weights(W: torch.Tensor, s: torch.Tensor, Wq=None, Ws=None, act_mult=None, stream=None):
@@ -164,8 +173,11 @@ def macaq_act_quant_plain(x: torch.Tensor, Aq=None, As=None, stream=None):
     return Aq, As
 
 
-def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: bool = False, stream=None):
-    """y = dec(A) dec(W)^T from MXFP4 operands; bf16 (default) or fp32 [M, N]."""
+def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: bool = False, workspace=None,
+                     data_parallel: bool = False, stream=None):
+    """y = dec(A) dec(W)^T from MXFP4 operands; bf16 (default) or fp32 [M, N].  A stream-K
+    workspace is allocated when not given (the schedule macaq_w4a4_linear uses);
+    data_parallel=True passes none (data-parallel schedule)."""
     _need(Aq, "Aq", torch.uint8, (M, K // 2))
     _need(Wq, "Wq", torch.uint8, (N, K // 2))
     _need(As, "As", torch.uint8)
@@ -173,8 +185,16 @@ def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: b
     dt = torch.float32 if out_fp32 else torch.bfloat16
     y = torch.empty(M, N, dtype=dt, device=Aq.device) if y is None else y
     _need(y, "y", dt, (M, N))
+    if data_parallel:
+        workspace = None
+    elif workspace is None:
+        workspace = torch.empty(max(gemm_workspace_bytes(M, N, K), 1), dtype=torch.uint8, device=Aq.device)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
     _check(load_library().macaq_mxfp4_gemm(_ptr(Aq), _ptr(As), M, _ptr(Wq), _ptr(Ws), N, K, _ptr(y),
-                                           1 if out_fp32 else 0, _stream(stream)), "macaq_mxfp4_gemm")
+                                           1 if out_fp32 else 0, _ptr(workspace),
+                                           0 if workspace is None else workspace.numel(), _stream(stream)),
+           "macaq_mxfp4_gemm")
     return y
 
 
@@ -188,7 +208,7 @@ def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor,
     _need(Ws, "Ws", torch.uint8)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
     _need(y, "y", torch.bfloat16, (M, N))
-    need = linear_workspace_bytes(M, K)
+    need = linear_workspace_bytes(M, N, K)
     workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
     _need(workspace, "workspace", torch.uint8)
     _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),

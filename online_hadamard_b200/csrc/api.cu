@@ -48,12 +48,6 @@ extern "C" int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K) {
     return scale_offset(r, kb, padded_blocks(K));
 }
 
-extern "C" size_t macaq_linear_workspace_bytes(int64_t M, int64_t K) {
-    if (check_shape(M, K) != MACAQ_OK) return 0;
-    const int64_t codes = ((M * (K / 2) + 255) / 256) * 256;
-    return static_cast<size_t>(codes + scale_bytes(M, K));
-}
-
 extern "C" int macaq_device_status(int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MACAQ_ECUDA;
     int v = 0;

@@ -13,12 +13,15 @@
 // Costs and rules of that array:
 //   * it is kNoAllocScratchBytes (32 MiB) on every GPU that loads the library, held until
 //     the process exits;
-//   * problems whose scratch (macaq_linear_workspace_bytes(M, K)) exceeds it are rejected
-//     with MACAQ_ETOOLARGE before anything is launched;
+//   * problems whose activation codes and scales exceed it are rejected with
+//     MACAQ_ETOOLARGE before anything is launched; what is left of the array after them
+//     serves as the GEMM's stream-K scratch when it is large enough, otherwise the GEMM
+//     runs its data-parallel schedule (same results up to fp32 summation order);
 //   * every call shares it and it keeps the previous call's contents.  Nothing in it has
 //     to start at zero: each call writes every code byte and every scale byte of its real
-//     rows before reading them, and the bytes it does not write (padded rows of the last
-//     128-row scale atom) only feed outputs that are never stored;
+//     rows before reading them, clears the stream-K flags before the GEMM reads them, and
+//     the bytes it does not write (padded rows of the last 128-row scale atom, stale
+//     partial sums) are never used for a stored output;
 //   * two calls whose kernels overlap on the GPU (different streams without ordering, or
 //     several host threads) race on the array and corrupt each other's results: order
 //     them on one stream or serialise them;
@@ -37,10 +40,6 @@ constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 // The scratch itself: static device memory, never allocated or freed at run time.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-int run_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq, const uint8_t* Ws,
-                   int64_t N, int64_t K, void* y, int y_fp32, cudaStream_t stream, bool pdl);
-int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
-                               uint8_t* Aq, uint8_t* As, cudaStream_t stream);
 
 // Device address of g_noalloc_scratch on the current device.  In host code the array's
 // name is only a host-side stand-in: a kernel given it would fault or, where the GPU can
@@ -74,12 +73,16 @@ extern "C" int macaq_w4a4_linear_noalloc(const uint16_t* x, int64_t M, int64_t K
     if (int st = check_shape(N, K)) return st;
     if (!aligned16(x) || !aligned16(act_mult) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y))
         return MACAQ_EALIGN;
-    if (macaq_linear_workspace_bytes(M, K) > kNoAllocScratchBytes) return MACAQ_ETOOLARGE;
+    const size_t act_bytes = linear_activation_bytes(M, K);
+    if (act_bytes > kNoAllocScratchBytes) return MACAQ_ETOOLARGE;
     uint8_t* scratch = nullptr;
     if (int st = noalloc_scratch(&scratch)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t* Aq = scratch;
-    uint8_t* As = Aq + ((M * (K / 2) + 255) / 256) * 256;
-    if (int rc = launch_act_transform_quant(x, M, K, act_mult, Aq, As, s)) return rc;
-    return run_mxfp4_gemm(Aq, As, M, Wq, Ws, N, K, y, 0, s, true);
+    const LinearWorkspace l = linear_workspace_layout(scratch, M, K);
+    const bool streamk = act_bytes + l.gemm_bytes <= kNoAllocScratchBytes;
+    if (int rc = launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, s, reinterpret_cast<uint32_t*>(l.gemm),
+                                            streamk ? gemm_ctas(M) : 0))
+        return rc;
+    const GemmScratch ws{streamk ? l.gemm : nullptr, streamk ? l.gemm_bytes : 0, false};
+    return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, s, true);
 }

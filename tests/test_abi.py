@@ -57,9 +57,8 @@ def test_size_helpers_reject_bad_shapes():
     assert mq.scale_bytes(0, 256) == 0
     assert mq.scale_bytes(4, 48) == 0
     assert mq.scale_offset(0, 8, 256) == -1
-    assert mq.linear_workspace_bytes(16, 33) == 0
-    ws = mq.linear_workspace_bytes(16, 256)
-    assert ws == 256 * ((16 * 128 + 255) // 256) + layout.scale_bytes(16, 256)
+    assert mq.linear_workspace_bytes(16, 64, 33) == 0
+    assert mq.gemm_workspace_bytes(0, 64, 32) == 0
 
 
 FAKE = 0x10000  # aligned, never dereferenced: every call below fails validation first
@@ -75,18 +74,16 @@ def test_validation_null_shape_alignment():
     P = ctypes.c_void_p
     # null pointers
     assert _call("macaq_act_transform_quant", None, 4, 64, P(FAKE), P(FAKE), P(FAKE), None) == -1
-    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, None, 0, None) == -1
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, None, 0, None, 0, None) == -1
     # shapes
     assert _call("macaq_act_transform_quant", P(FAKE), 4, 48, P(FAKE), P(FAKE), P(FAKE), None) == -2
     assert _call("macaq_act_quant_plain", P(FAKE), 0, 64, P(FAKE), P(FAKE), None) == -2
-    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 0, 64, P(FAKE), 0, None) == -2
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 0, 64, P(FAKE), 0, None, 0, None) == -2
     assert _call("macaq_fold_weights", P(FAKE), 8, 16, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None) == -2
     # alignment
     assert _call("macaq_act_transform_quant", P(MIS), 4, 64, P(FAKE), P(FAKE), P(FAKE), None) == -3
-    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(MIS), 0, None) == -3
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(MIS), 0, None, 0, None) == -3
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(FAKE), 0, P(MIS), 1 << 30,
+                 None) == -3
     # bad flag
-    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(FAKE), 2, None) == -1
-    # workspace too small
-    need = mq.linear_workspace_bytes(4, 64)
-    assert _call("macaq_w4a4_linear", P(FAKE), 4, 64, P(FAKE), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE),
-                 need - 1, None) == -6
+    assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(FAKE), 2, None, 0, None) == -1

@@ -8,7 +8,8 @@ codes and scales exactly in fp64.  Gates (relative Frobenius error):
 The error of the bf16 output against the unrounded exact result is dominated by bf16's 8
 significand bits (~1.5e-3 relative RMS); it is reported, not gated.
 Shapes span several tiles with ragged M, N and K tails, both kernel orientations (swap-AB
-for M <= 128, 128x256 tiles above) and every MMA-N width."""
+for M <= 128, 128x256 tiles above), every MMA-N width, and both schedules: stream-K (tiles
+split across CTAs, fp32 partials added by the tile's owner) and data-parallel."""
 import numpy as np
 import pytest
 import torch
@@ -47,6 +48,9 @@ SHAPES = [
     (1, 256, 256), (1, 7, 32), (4, 136, 96), (16, 384, 512), (17, 200, 288), (33, 520, 800),
     (64, 256, 1024), (65, 130, 256), (100, 1000, 800), (128, 128, 256), (129, 300, 320),
     (256, 512, 512), (300, 520, 1056), (511, 777, 640), (1024, 2048, 2048),
+    # long K, few tiles: stream-K splits every tile across many CTAs (owner + ~10-18
+    # contributors), swap-AB and 128 x 256 orientations
+    (16, 2048, 8192), (200, 1024, 8192), (70, 1100, 6144),
 ]
 
 
@@ -59,8 +63,11 @@ def test_gemm_identical_codes(mq, M, N, K):
     Wg, Wsg = to_device_mx(Wc, Ws, N, K)
     y32 = mq.macaq_mxfp4_gemm(Ag, Asg, Wg, Wsg, M, N, K, out_fp32=True)
     y16 = mq.macaq_mxfp4_gemm(Ag, Asg, Wg, Wsg, M, N, K)
+    y32dp = mq.macaq_mxfp4_gemm(Ag, Asg, Wg, Wsg, M, N, K, out_fp32=True, data_parallel=True)
     torch.cuda.synchronize()
     ref = oracle.mx_gemm(Ac, As, Wc, Ws)
+    # both schedules (stream-K fix-up and data-parallel) meet the gate
+    assert gu.rel_fro(gu.to_np(y32dp), ref) <= TOL
     e32 = gu.rel_fro(gu.to_np(y32), ref)
     e16 = gu.rel_fro(gu.to_np(y16.float()), gu.bf16_round(ref))
     e16_raw = gu.rel_fro(gu.to_np(y16.float()), ref)

@@ -66,11 +66,11 @@ def test_linear_workspace_and_errors(mq):
     s = torch.ones(K, device="cuda")
     Wq, Ws, am = mq.macaq_fold_weights(W, s)
     x = torch.randn(M, K, device="cuda").to(torch.bfloat16)
-    small = torch.empty(mq.linear_workspace_bytes(M, K) - 16, dtype=torch.uint8, device="cuda")
+    small = torch.empty(mq.linear_workspace_bytes(M, N, K) - 16, dtype=torch.uint8, device="cuda")
     with pytest.raises(mq.MacaqError) as ei:
         mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=small)
     assert ei.value.status == -6
-    ws = torch.full((mq.linear_workspace_bytes(M, K),), 0xFF, dtype=torch.uint8, device="cuda")
+    ws = torch.full((mq.linear_workspace_bytes(M, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
     y1 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=ws)
     y2 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N)
     assert torch.equal(y1, y2)

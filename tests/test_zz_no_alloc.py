@@ -70,7 +70,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch(mq):
     lib = mq.load_library()
     K = 8192
     M = 8192  # needs 32 MiB of codes plus scales: over the limit
-    assert mq.linear_workspace_bytes(M, K) > mq.NOALLOC_SCRATCH_BYTES
+    assert M * K // 2 + mq.scale_bytes(M, K) > mq.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x10000)  # validation fails before any pointer is used
     st = lib.macaq_w4a4_linear_noalloc(fake, M, K, fake, fake, fake, 64, fake, None)
     assert st == -7, mq.status_str(st)
