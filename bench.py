@@ -11,7 +11,7 @@ between two uses of a copy exceed the 126 MB L2, so every step streams from HBM.
 
 Printed on rank 0: one JSON line with the whole-job TFLOP/s, the roofline of the dominant
 kernel (the tcgen05 GEMM, timed live with CUDA events), the online-transform overhead over
-plain MXFP4 (plain quantisation + the same GEMM) and over the GEMM alone, an end-to-end
+plain MXFP4 (macaq_mxfp4_linear: plain quantisation + the same GEMM) and over the GEMM alone, an end-to-end
 figure through the C ABI with host buffers, the oracle's CPU throughput on a bounded
 sample, SM clocks sampled during the timed region, and secondary workloads (decode and
 the Qwen3-32B-shaped down projection).
@@ -186,10 +186,9 @@ class Layer:
                                  y=self.y[c], workspace=self.gws[c])
 
     def plain(self, i):
+        """Pure MXFP4: the same kernels as linear() without the scale and the transform."""
         c = i % self.copies
-        self.mq.macaq_act_quant_plain(self.x[c], Aq=self.Aq[c], As=self.As[c])
-        self.mq.macaq_mxfp4_gemm(self.Aq[c], self.As[c], self.Wq[c], self.Ws[c], self.wl.M, self.wl.N, self.wl.K,
-                                 y=self.y[c], workspace=self.gws[c])
+        self.mq.macaq_mxfp4_linear(self.x[c], self.Wq[c], self.Ws[c], self.wl.N, y=self.y[c], workspace=self.ws[c])
 
     def transform_only(self, i):
         c = i % self.copies
@@ -394,7 +393,7 @@ def main():
     ms_e2e = max_over_ranks(time_eager(layer.e2e, e2e_steps, 3, device))
     gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
     xform_bytes = wl.M * wl.K * 2 + wl.M * wl.K * (0.5 + 1 / 32) + wl.K * 4
-    traffic = recorded_traffic("mxf4_gemm_128x256:" + wl.name)
+    traffic = recorded_traffic("mxf4_gemm_pair_256x256:" + wl.name)
 
     extra = {}
     if not args.no_extra:
@@ -412,7 +411,7 @@ def main():
             "dtype": "mxfp4 (e2m1 x e2m1, ue8m0 scales, fp32 accumulate, bf16 out)", "data": "synthetic",
             "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {layer.copies} copies (> 3x L2)"},
-            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_kernel<256,4,false>", "achieved": gemm_tflops,
+            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<5> (2-CTA 256x256 tiles)", "achieved": gemm_tflops,
                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
                          "ms_per_launch": ms_gemm},

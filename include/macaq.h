@@ -85,9 +85,9 @@ int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
  * and the device's SM count). */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
-/* Bytes of scratch macaq_w4a4_linear needs on the current device: the activations' MXFP4
- * codes (M*K/2) and scales (macaq_scale_bytes(M, K)), each rounded up to 256, then
- * macaq_gemm_workspace_bytes(M, N, K). */
+/* Bytes of scratch macaq_w4a4_linear (and macaq_mxfp4_linear) needs on the current device:
+ * the activations' MXFP4 codes (M*K/2) and scales (macaq_scale_bytes(M, K)), each rounded
+ * up to 256, then macaq_gemm_workspace_bytes(M, N, K). */
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -120,8 +120,11 @@ int macaq_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const flo
  * macaq_w4a4_linear -- the layer's forward pass, y = x W^T computed as
  * MXFP4(x diag(act_mult) H) . MXFP4(W')^T (Abstract; the 2.3% end-to-end overhead over
  * plain MXFP4 quoted there is for this online transform): the activation transform and
- * quantisation run as the GEMM's prologue, the block-scaled MXFP4 x MXFP4 contraction
- * runs on the tensor cores with fp32 accumulation, and y is rounded to bf16 (RNE).
+ * MXFP4 quantisation kernel writes the activations' codes and scales into the workspace,
+ * then the block-scaled MXFP4 x MXFP4 GEMM (launched as a programmatic dependent of it)
+ * contracts them on the tensor cores with fp32 accumulation and rounds y to bf16 (RNE).
+ * Codes, scales and y are identical to those of macaq_act_transform_quant followed by
+ * macaq_mxfp4_gemm with a workspace.
  *   x         in   bf16 [M][K];  act_mult in fp32 [K]
  *   Wq, Ws    in   folded weights from macaq_fold_weights (N rows)
  *   y         out  bf16 [M][N]
@@ -138,6 +141,10 @@ int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_
  * the online transform against "pure MXFP4", Abstract).
  *
  * macaq_act_quant_plain: MXFP4 quantisation of x with no scale and no transform.
+ * macaq_mxfp4_linear: the plain MXFP4 linear layer, y = dec(MXFP4(x)) dec(Wq)^T in bf16,
+ *   run exactly like macaq_w4a4_linear (same kernels, same workspace size and rules)
+ *   without the per-channel scale and the Hadamard transform: the "pure MXFP4" against
+ *   which the transform's overhead is measured.
  * macaq_mxfp4_gemm: y = dec(A) dec(W)^T for already-quantised operands, fp32 accumulate;
  *   y is bf16 [M][N] (y_is_fp32 = 0) or fp32 [M][N] (y_is_fp32 = 1).  With a workspace of
  *   macaq_gemm_workspace_bytes(M, N, K) the GEMM balances its last wave with a stream-K
@@ -147,6 +154,8 @@ int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_
  */
 int macaq_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                           void* stream);
+int macaq_mxfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wq, const uint8_t* Ws,
+                       int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes, void* stream);
 int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
                      const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32,
                      void* workspace, size_t workspace_bytes, void* stream);

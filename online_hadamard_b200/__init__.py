@@ -24,8 +24,8 @@ from . import build as _build_mod
 __all__ = [
     "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes", "gemm_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
-    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_w4a4_linear_noalloc", "macaq_device_status", "status_str",
-    "EXPORTED_SYMBOLS",
+    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_linear_noalloc",
+    "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
 # Every symbol include/macaq.h declares.
@@ -33,7 +33,8 @@ EXPORTED_SYMBOLS = (
     "macaq_status_str", "macaq_scale_bytes", "macaq_scale_offset", "macaq_linear_workspace_bytes",
     "macaq_gemm_workspace_bytes",
     "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
-    "macaq_act_quant_plain", "macaq_mxfp4_gemm", "macaq_device_status", "macaq_w4a4_linear_noalloc",
+    "macaq_act_quant_plain", "macaq_mxfp4_linear", "macaq_mxfp4_gemm", "macaq_device_status",
+    "macaq_w4a4_linear_noalloc",
 )
 
 MACAQ_OK = 0
@@ -74,10 +75,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_act_quant_plain.argtypes = [p, i64, i64, p, p, p]
         lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p, sz, p]
         lib.macaq_w4a4_linear.argtypes = [p, i64, i64, p, p, p, i64, p, p, sz, p]
+        lib.macaq_mxfp4_linear.argtypes = [p, i64, i64, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
         lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
         for name in ("macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
-                     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_device_status",
+                     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_linear_noalloc"):
             getattr(lib, name).restype = i32
         if path is None:
@@ -125,7 +127,7 @@ def scale_offset(r: int, kb: int, K: int) -> int:
 
 
 def linear_workspace_bytes(M: int, N: int, K: int) -> int:
-    """Scratch bytes macaq_w4a4_linear needs on the current device."""
+    """Scratch bytes macaq_w4a4_linear and macaq_mxfp4_linear need on the current device."""
     return int(load_library().macaq_linear_workspace_bytes(M, N, K))
 
 
@@ -214,6 +216,23 @@ def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor,
     _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
                                             _ptr(workspace), workspace.numel(), _stream(stream)),
            "macaq_w4a4_linear")
+    return y
+
+
+def macaq_mxfp4_linear(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int, y=None, workspace=None,
+                       stream=None):
+    """Plain MXFP4 linear (no scale, no transform): the baseline of the transform's overhead."""
+    M, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2))
+    _need(Ws, "Ws", torch.uint8)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N))
+    need = linear_workspace_bytes(M, N, K)
+    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8)
+    _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
+                                             workspace.numel(), _stream(stream)), "macaq_mxfp4_linear")
     return y
 
 

@@ -40,6 +40,8 @@ namespace macaq {
 
 int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
                                uint8_t* Aq, uint8_t* As, cudaStream_t stream, uint32_t* clear, int clear_words);
+int launch_act_quant_plain_clear(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
+                                 cudaStream_t stream, uint32_t* clear, int clear_words);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -163,14 +165,15 @@ struct Work {
 };
 
 struct WorkIter {
-    int dp_next;
+    int dp_next, id, count;
     int64_t pos, hi;
 
-    __device__ __forceinline__ explicit WorkIter(const GemmParams& p) {
-        dp_next = blockIdx.x;
-        const int64_t G = gridDim.x;
-        pos = p.sk_units * blockIdx.x / G;
-        hi = p.sk_units * (blockIdx.x + 1) / G;
+    // `id` of `count` scheduling units: the CTA for the one-CTA kernel, the CTA pair for the
+    // pair kernel (both CTAs of a pair walk the same items).
+    __device__ __forceinline__ WorkIter(const GemmParams& p, int id_, int count_) : id(id_), count(count_) {
+        dp_next = id;
+        pos = p.sk_units * id / count;
+        hi = p.sk_units * (id + 1) / count;
     }
 
     __device__ __forceinline__ bool next(const GemmParams& p, Work& w) {
@@ -181,7 +184,7 @@ struct WorkIter {
             w.k1 = KT;
             w.kind = kFull;
             w.c_last = 0;
-            dp_next += gridDim.x;
+            dp_next += count;
             return true;
         }
         if (pos >= hi) return false;
@@ -195,9 +198,9 @@ struct WorkIter {
             w.kind = kFull;
         } else if (w.k0 == 0) {
             w.kind = kOwner;
-            // last CTA whose range holds a unit of this tile: max c with U c / G <= t0 + KT - 1
-            const int64_t U = p.sk_units, G = gridDim.x;
-            w.c_last = static_cast<int>(((t0 + KT) * G + U - 1) / U - 1);
+            // last unit whose range holds a K step of this tile: max c with U c / count <= t0 + KT - 1
+            const int64_t U = p.sk_units;
+            w.c_last = static_cast<int>(((t0 + KT) * count + U - 1) / U - 1);
         } else {
             w.kind = kPartial;
         }
@@ -210,6 +213,94 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Per-thread state of an epilogue thread for one work item.
+struct EpiCtx {
+    int etid, lane, warp;
+    int unit, units;              // scheduling unit of this CTA (CTA or pair) and their number
+    int slot_self;                // this CTA's partial-sum slot
+    int slot_stride, slot_off;    // contributor unit c -> its slot c * slot_stride + slot_off
+    int64_t prow;                 // output row (P side) of this thread
+    int64_t row0;                 // first output row of this warp's 32 rows
+    int64_t q0;                   // first output column (Q side) of this warp's half of the tile
+    uint8_t* staging;             // this warp's 2 KB output staging buffer (TMA-store path)
+};
+
+// After the accumulator of `w` is in registers (v = this thread's BN/2 fp32 columns): write a
+// stream-K partial, or add the contributors' partials (owner), then store y.
+template <int BN, bool SWAP>
+__device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtensorMap* tmap_y, const Work& w,
+                                            const EpiCtx& e, uint32_t* v, int& abort) {
+    constexpr int kHalf = BN / 2;
+    constexpr int kChunk = kHalf >= 32 ? 32 : kHalf;
+    if (w.kind == kPartial) {
+        // fp32 partial to this CTA's slot, [chunk of 4 columns][epilogue thread]; the slot's
+        // counter reaches kEpiThreads once every thread's part is visible
+        float4* slot = reinterpret_cast<float4*>(prm.partials + static_cast<int64_t>(e.slot_self) * (kBM * BN));
+#pragma unroll
+        for (int j = 0; j < kHalf / 4; ++j)
+            __stcg(slot + j * kEpiThreads + e.etid,
+                   make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+        __threadfence();
+        atomicAdd(prm.flags + e.slot_self, 1u);
+        return;
+    }
+    if (w.kind == kOwner) {
+        const int64_t U = prm.sk_units, G = e.units;
+        for (int c = e.unit + 1; c <= w.c_last; ++c) {
+            if (U * c / G == U * (c + 1) / G) continue;  // empty range: no partial
+            const int slot_id = c * e.slot_stride + e.slot_off;
+            if (!abort) {
+                const long long t0 = clock64();
+                while (ld_acquire(prm.flags + slot_id) < static_cast<uint32_t>(kEpiThreads)) {
+                    if (clock64() - t0 > kWaitLimitCycles) {
+                        atomicExch(&g_device_status, MACAQ_ETIMEOUT);
+                        abort = 1;
+                        break;
+                    }
+                }
+            }
+            const float4* slot = reinterpret_cast<const float4*>(prm.partials + static_cast<int64_t>(slot_id) * (kBM * BN));
+#pragma unroll
+            for (int j = 0; j < kHalf / 4; ++j) {
+                const float4 q = __ldcg(slot + j * kEpiThreads + e.etid);
+                v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + q.x);
+                v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + q.y);
+                v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q.z);
+                v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q.w);
+            }
+        }
+    }
+    if constexpr (!SWAP && kHalf % 32 == 0) {
+        if (prm.tma_store) {
+            // bf16 tile through this warp's 2 KB staging buffer (32 rows x 64 B, 64-byte
+            // swizzle: conflict-free 16-byte writes) and a TMA store per 32 columns; the
+            // store clips rows and columns past the matrix edge.
+#pragma unroll
+            for (int c = 0; c < kHalf; c += 32) {
+                if (e.lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
+                __syncwarp();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t* r = v + c + 8 * q4;
+                    *reinterpret_cast<uint4*>(e.staging + e.lane * 64 + 16 * (q4 ^ ((e.lane >> 1) & 3))) =
+                        make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                                   pack_bf16x2(r[6], r[7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (e.lane == 0) {
+                    tma_store_2d(tmap_y, e.staging, static_cast<int32_t>(e.q0 + c), static_cast<int32_t>(e.row0));
+                    bulk_commit_group();
+                }
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < kHalf; c += kChunk) store_chunk<kChunk, SWAP>(prm, e.prow, e.q0 + c, v + c);
 }
 
 template <int BN, int STAGES, bool SWAP>
@@ -259,7 +350,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             griddep_wait();  // operands may come from the kernel launched just before
             int stage = 0;
             uint32_t phase = 0;
-            WorkIter it(prm);
+            WorkIter it(prm, blockIdx.x, gridDim.x);
             Work w;
             while (!abort && it.next(prm, w)) {
                 const int pt = w.tile % prm.num_p_tiles;
@@ -298,15 +389,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             uint32_t sfbuf = 0;
-            WorkIter it(prm);
+            WorkIter it(prm, blockIdx.x, gridDim.x);
             Work w;
             while (!abort && it.next(prm, w)) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, &abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * Cfg::kAccStride;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
+                    // the TMA data of the stage is complete once the barrier phase flips; no
+                    // tcgen05 fence here (it would drain the MMA queue every K step)
                     if (!mbar_wait(&full[stage], phase, &abort)) break;
-                    tc_fence_after();
                     const uint32_t sp = smem_u32(smem + stage * Cfg::kStageBytes);
                     const uint32_t sq = sp + Cfg::kPBytes;
                     const uint32_t ssfp = sq + Cfg::kQBytes;
@@ -353,7 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int etid = threadIdx.x - 64;       // 0..255 among the epilogue threads
         int acc = 0;
         uint32_t acc_phase = 0;
-        WorkIter it(prm);
+        WorkIter it(prm, blockIdx.x, gridDim.x);
         Work w;
         if (prm.sk_units > 0) griddep_wait();  // the flags were cleared by the kernel launched before
         while (!abort && it.next(prm, w)) {
@@ -374,74 +466,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 acc = 0;
                 acc_phase ^= 1u;
             }
-            if (w.kind == kPartial) {
-                // fp32 partial to this CTA's slot, [chunk of 4 columns][epilogue thread]; the
-                // slot's counter reaches kEpiThreads once every thread's part is visible
-                float4* slot = reinterpret_cast<float4*>(prm.partials + static_cast<int64_t>(blockIdx.x) * (kBM * BN));
-#pragma unroll
-                for (int j = 0; j < kHalf / 4; ++j)
-                    __stcg(slot + j * kEpiThreads + etid,
-                           make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                       __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
-                __threadfence();
-                atomicAdd(prm.flags + blockIdx.x, 1u);
-                continue;
-            }
-            if (w.kind == kOwner) {
-                const int64_t U = prm.sk_units, G = gridDim.x;
-                for (int c = blockIdx.x + 1; c <= w.c_last; ++c) {
-                    if (U * c / G == U * (c + 1) / G) continue;  // empty range: no partial
-                    if (!abort) {
-                        const long long t0 = clock64();
-                        while (ld_acquire(prm.flags + c) < static_cast<uint32_t>(kEpiThreads)) {
-                            if (clock64() - t0 > kWaitLimitCycles) {
-                                atomicExch(&g_device_status, MACAQ_ETIMEOUT);
-                                abort = 1;
-                                break;
-                            }
-                        }
-                    }
-                    const float4* slot = reinterpret_cast<const float4*>(prm.partials + static_cast<int64_t>(c) * (kBM * BN));
-#pragma unroll
-                    for (int j = 0; j < kHalf / 4; ++j) {
-                        const float4 q = __ldcg(slot + j * kEpiThreads + etid);
-                        v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + q.x);
-                        v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + q.y);
-                        v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q.z);
-                        v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q.w);
-                    }
-                }
-            }
-            const int64_t q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
-            if constexpr (!SWAP && kHalf % 32 == 0) {
-                if (prm.tma_store) {
-                    // bf16 tile through this warp's 2 KB staging buffer (32 rows x 64 B, 64-byte
-                    // swizzle: conflict-free 16-byte writes) and a TMA store per 32 columns;
-                    // the store clips rows and columns past the matrix edge.
-                    uint8_t* stg = staging + (warp - 2) * 2048;
-#pragma unroll
-                    for (int c = 0; c < kHalf; c += 32) {
-                        if (lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
-                        __syncwarp();
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const uint32_t* r = v + c + 8 * q4;
-                            *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
-                                make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
-                                           pack_bf16x2(r[6], r[7]));
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmap_y, stg, static_cast<int32_t>(q0 + c), pt * kBM + sub * 32);
-                            bulk_commit_group();
-                        }
-                    }
-                    continue;
-                }
-            }
-#pragma unroll
-            for (int c = 0; c < kHalf; c += kChunk) store_chunk<kChunk, SWAP>(prm, prow, q0 + c, v + c);
+            EpiCtx e;
+            e.etid = etid;
+            e.lane = lane;
+            e.warp = warp;
+            e.unit = blockIdx.x;
+            e.units = gridDim.x;
+            e.slot_self = blockIdx.x;
+            e.slot_stride = 1;
+            e.slot_off = 0;
+            e.prow = prow;
+            e.row0 = static_cast<int64_t>(pt) * kBM + sub * 32;
+            e.q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
+            e.staging = staging + (warp - 2) * 2048;
+            finish_item<BN, SWAP>(prm, &tmap_y, w, e, v, abort);
         }
         if (lane == 0) bulk_wait_group<0>();  // output stores complete before the CTA exits
     }
@@ -450,6 +488,214 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel
+//
+// Prefill tiles of 256 x 256 on a cluster of two CTAs (the two SMs of a TPC) sharing one
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64):
+//   - each CTA TMA-loads its own 128 rows of the activation tile and its own 128 rows of the
+//     weight tile per K step, so a weight panel crosses L2 -> SM once per pair instead of once
+//     per CTA (35 KB per CTA per K step instead of 51 KB);
+//   - each CTA loads the scales of its 128 activation rows and of all 256 weight rows;
+//     tcgen05.cp.cta_group::2 moves them into the same TMEM columns of both CTAs;
+//   - all loads of both CTAs complete on the even CTA's "full" barrier; its single MMA thread
+//     issues the pair MMAs and multicasts each stage's release to both CTAs' "empty" barriers
+//     and each tile's completion to both "acc_full" barriers;
+//   - each CTA's eight epilogue warps drain its 128 accumulator rows and release them on the
+//     even CTA's "acc_empty" barrier (512 arrivals: both CTAs).
+// Scheduling (data-parallel waves then stream-K) works on pairs; partial-sum slots stay per CTA.
+constexpr int kPairStages = 5;
+struct PairCfg {
+    static constexpr int kABytes = 128 * kStageKBytes;     // this CTA's 128 activation rows
+    static constexpr int kBBytes = 128 * kStageKBytes;     // this CTA's 128 weight rows
+    static constexpr int kSFABytes = 1024;                 // 128 rows x 8 blocks
+    static constexpr int kSFBBytes = 2048;                 // all 256 weight rows x 8 blocks
+    static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+    static constexpr int kSFBufCols = 8 + 16;              // SFA 2 groups x 4, SFB 2 groups x 8
+    static constexpr int kSFBase = 256;                    // after the 256-column accumulator
+    static constexpr int kTmemCols = 512;
+    static_assert(kStageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
+    static_assert(kSFBase + 2 * kSFBufCols <= kTmemCols, "tensor memory budget");
+};
+
+template <int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                          const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                          const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm) {
+    using Cfg = PairCfg;
+    constexpr int BN = 256;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* staging = smem + STAGES * Cfg::kStageBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * kEpiThreads);
+        fence_mbar_init();
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+        prefetch_tmap(&tmap_sfa);
+        prefetch_tmap(&tmap_sfb);
+        if (prm.tma_store) prefetch_tmap(&tmap_y);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers and tensor memory exist before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    int abort = 0;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------- producer (both CTAs)
+            griddep_wait();
+            int stage = 0;
+            uint32_t phase = 0;
+            WorkIter it(prm, pair, pairs);
+            Work w;
+            while (!abort && it.next(prm, w)) {
+                const int pt = w.tile / prm.num_q_tiles;  // activation-block major: early tiles need early rows
+                const int qt = w.tile % prm.num_q_tiles;
+                const int a_row = pt * 256 + static_cast<int>(rank) * 128;
+                const int b_row = qt * 256 + static_cast<int>(rank) * 128;
+                for (int kt = w.k0; kt < w.k1; ++kt) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
+                    uint8_t* sb = smem + stage * Cfg::kStageBytes;
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+                    tma_load_2d_pair(sb, &tmap_a, kt * kStageKBytes, a_row, &full[stage]);
+                    tma_load_2d_pair(sb + Cfg::kABytes, &tmap_b, kt * kStageKBytes, b_row, &full[stage]);
+                    uint8_t* sf = sb + Cfg::kABytes + Cfg::kBBytes;
+                    // scale atoms: 1 KB (two 512-byte atoms) per 128 rows per K step, as uint32 boxes
+                    tma_load_2d_pair(sf, &tmap_sfa, kt * 256, 2 * pt + static_cast<int>(rank), &full[stage]);
+                    tma_load_2d_pair(sf + 1024, &tmap_sfb, kt * 256, 2 * qt, &full[stage]);
+                    tma_load_2d_pair(sf + 2048, &tmap_sfb, kt * 256, 2 * qt + 1, &full[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (even CTA only)
+            const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) | (1u << 23) |
+                                   (static_cast<uint32_t>(256 >> 4) << 24);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t acc_phase = 0;
+            uint32_t sfbuf = 0;
+            WorkIter it(prm, pair, pairs);
+            Work w;
+            while (!abort && it.next(prm, w)) {
+                if (!mbar_wait(acc_empty, acc_phase ^ 1u, &abort)) break;
+                acc_phase ^= 1u;
+                tc_fence_after();
+                for (int kt = w.k0; kt < w.k1; ++kt) {
+                    if (!mbar_wait(&full[stage], phase, &abort)) break;  // no tcgen05 fence: see above
+                    const uint32_t sp = smem_u32(smem + stage * Cfg::kStageBytes);
+                    const uint32_t sq = sp + Cfg::kABytes;
+                    const uint32_t ssfa = sq + Cfg::kBBytes;
+                    const uint32_t ssfb = ssfa + Cfg::kSFABytes;
+                    const uint32_t tsfa = tmem_base + Cfg::kSFBase + sfbuf * Cfg::kSFBufCols;
+                    const uint32_t tsfb = tsfa + 8;
+                    sfbuf ^= 1u;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        tc_cp_sf_pair(tsfa + 4 * g, desc_sf(ssfa + 512 * g));
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) tc_cp_sf_pair(tsfb + 8 * g + 4 * i, desc_sf(ssfb + 1024 * i + 512 * g));
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t g = j >> 1;
+                        const uint32_t id = (j & 1) * 2;
+                        const uint32_t sfa = (tsfa + 4 * g) | (id << 30);
+                        const uint32_t sfb = (tsfb + 8 * g) | (id << 30);
+                        tc_mma_mxf4_pair(tmem_base, desc_sw128(sp + 32 * j), desc_sw128(sq + 32 * j),
+                                         idesc | (id << 29) | (id << 4), sfa, sfb, (kt != w.k0 || j != 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(&empty[stage]);  // frees the stage in both CTAs
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                tc_commit_pair(acc_full);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------------- epilogue (both CTAs)
+        constexpr int kHalf = BN / 2;
+        const int sub = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int etid = threadIdx.x - 64;
+        uint32_t acc_phase = 0;
+        WorkIter it(prm, pair, pairs);
+        Work w;
+        if (prm.sk_units > 0) griddep_wait();
+        while (!abort && it.next(prm, w)) {
+            const int pt = w.tile / prm.num_q_tiles;  // activation-block major: early tiles need early rows
+            const int qt = w.tile % prm.num_q_tiles;
+            if (!mbar_wait(acc_full, acc_phase, &abort)) break;
+            acc_phase ^= 1u;
+            tc_fence_after();
+            const int64_t row0 = static_cast<int64_t>(pt) * 256 + rank * 128 + sub * 32;
+            const uint32_t tbase = tmem_base + half * kHalf + (static_cast<uint32_t>(sub * 32) << 16);
+            uint32_t v[kHalf];
+#pragma unroll
+            for (int c = 0; c < kHalf; c += 32) tmem_ld_cols<32>(tbase + c, v + c);
+            tmem_ld_wait();
+            tc_fence_before();
+            if (leader)
+                mbar_arrive(acc_empty);
+            else
+                mbar_arrive_cluster(acc_empty, 0);
+            EpiCtx e;
+            e.etid = etid;
+            e.lane = lane;
+            e.warp = warp;
+            e.unit = pair;
+            e.units = pairs;
+            e.slot_self = blockIdx.x;
+            e.slot_stride = 2;
+            e.slot_off = static_cast<int>(rank);
+            e.prow = row0 + lane;
+            e.row0 = row0;
+            e.q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
+            e.staging = staging + (warp - 2) * 2048;
+            finish_item<BN, false>(prm, &tmap_y, w, e, v, abort);
+        }
+        if (lane == 0) bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer's shared memory and tensor memory are no longer in use
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
 }
 
 // --------------------------------------------------------------------------- host side
@@ -482,6 +728,23 @@ static bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows,
     return r == CUDA_SUCCESS;
 }
 
+// Tensor map of an E8M0 scale buffer in the MMA tile layout, viewed as uint32 [row blocks]
+// [KBp * 32]: one box = 256 words = the two 512-byte atoms of one 128-row block for one
+// 256-element K step.
+static bool make_sf_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t K) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return false;
+    const int64_t kbp = padded_blocks(K);
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kbp * 32), static_cast<cuuint64_t>((rows + 127) / 128)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kbp * 128)};
+    cuuint32_t box[2] = {256, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(scales), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int BN, int STAGES, bool SWAP>
 static int smem_bytes() {
     return STAGES * TileCfg<BN>::kStageBytes + (SWAP ? 0 : kStagingBytes) + (2 * STAGES + 4) * 8 + 16 + 1024;
@@ -501,9 +764,30 @@ static bool make_out_map(CUtensorMap* map, void* y, int64_t rows, int64_t cols) 
     return r == CUDA_SUCCESS;
 }
 
+// Per-device cache of a launch-configuration query (the answers depend only on the device).
+template <class F>
+static int cached_per_device(int (&cache)[64], F&& query) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return query();
+    if (cache[dev] == 0) {
+        const int v = query();
+        cache[dev] = v > 0 ? v : -1;
+    }
+    return cache[dev] > 0 ? cache[dev] : 0;
+}
+
 // CTAs of the persistent grid: SMs x resident CTAs per SM (shared memory and TMEM permitting).
 template <int BN, int STAGES, bool SWAP>
+static int grid_ctas_query();
+
+template <int BN, int STAGES, bool SWAP>
 static int grid_ctas() {
+    static int cache[64] = {0};
+    return cached_per_device(cache, [] { return grid_ctas_query<BN, STAGES, SWAP>(); });
+}
+
+template <int BN, int STAGES, bool SWAP>
+static int grid_ctas_query() {
     auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP>;
     const int smem = smem_bytes<BN, STAGES, SWAP>();
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
@@ -609,6 +893,108 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
 
 // Kernel configuration for M rows of activations: swap-AB with the narrowest N that holds
 // the tokens for M <= 128, 128 x 256 tiles above.  `f` is called with the configuration.
+static int pair_smem_bytes() {
+    return kPairStages * PairCfg::kStageBytes + kStagingBytes + (2 * kPairStages + 2) * 8 + 16 + 1024;
+}
+
+static int gemm_pairs_query();
+
+// CTA pairs that can be resident at once (two SMs of a TPC each); 0 if cluster launch fails.
+static int gemm_pairs() {
+    static int cache[64] = {0};
+    return cached_per_device(cache, [] { return gemm_pairs_query(); });
+}
+
+static int gemm_pairs_query() {
+    auto kernel = mxf4_gemm_pair_kernel<kPairStages>;
+    const int smem = pair_smem_bytes();
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sm_count() & ~1));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return clusters;
+}
+
+static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int pairs, cudaStream_t stream, bool pdl) {
+    CUtensorMap ma, mb, msa, msb, my;
+    if (!make_codes_map(&ma, op.pq, op.p_rows, op.K, 128) || !make_codes_map(&mb, op.qq, op.q_rows, op.K, 128) ||
+        !make_sf_map(&msa, op.ps, op.p_rows, op.K) || !make_sf_map(&msb, op.qs, op.q_rows, op.K))
+        return MACAQ_ECUDA;
+    GemmParams prm;
+    prm.sf_p = op.ps;
+    prm.sf_q = op.qs;
+    prm.p_rows = op.p_rows;
+    prm.q_rows = op.q_rows;
+    prm.K = op.K;
+    prm.kbp = padded_blocks(op.K);
+    prm.y = op.y;
+    prm.ldy = op.ldy;
+    prm.y_fp32 = op.y_fp32;
+    prm.num_p_tiles = static_cast<int>((op.p_rows + 255) / 256);
+    prm.num_q_tiles = static_cast<int>((op.q_rows + 255) / 256);
+    prm.num_k_tiles = static_cast<int>((op.K + kStageK - 1) / kStageK);
+    prm.q_row_blocks = static_cast<int>((op.q_rows + 127) / 128);
+    prm.tma_store = (!op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
+    if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows)) return MACAQ_ECUDA;
+    if (!prm.tma_store) my = ma;  // unused placeholder
+
+    const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
+    const int64_t rounds_dp = (tiles + pairs - 1) / pairs;
+    const int64_t saved_steps = (rounds_dp * pairs - tiles) * prm.num_k_tiles / pairs;
+    const bool streamk = ws.ptr != nullptr && ws.bytes >= streamk_bytes<256>(2 * pairs) && tiles % pairs != 0 &&
+                         prm.num_k_tiles > 1 && saved_steps >= streamk_cost_steps<256>();
+    int64_t grid_pairs = pairs;
+    if (streamk) {
+        const int64_t full_waves = tiles / pairs;
+        prm.dp_tiles = static_cast<int>((full_waves > 0 ? full_waves - 1 : 0) * pairs);
+        prm.sk_units = (tiles - prm.dp_tiles) * static_cast<int64_t>(prm.num_k_tiles);
+        if (grid_pairs > prm.sk_units) grid_pairs = prm.sk_units;
+        const int ctas = 2 * pairs;
+        prm.flags = static_cast<uint32_t*>(ws.ptr);
+        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + ((ctas * 4 + 255) / 256) * 256);
+        if (ws.clear_flags && cudaMemsetAsync(prm.flags, 0, sizeof(uint32_t) * ctas, stream) != cudaSuccess)
+            return MACAQ_ECUDA;
+    } else {
+        if (grid_pairs > tiles) grid_pairs = tiles;
+        prm.dp_tiles = static_cast<int>(tiles);
+        prm.sk_units = 0;
+        prm.flags = nullptr;
+        prm.partials = nullptr;
+    }
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * grid_pairs));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    if (cudaLaunchKernelEx(&cfg, mxf4_gemm_pair_kernel<kPairStages>, ma, mb, msa, msb, my, prm) != cudaSuccess)
+        return MACAQ_ECUDA;
+    return launch_status();
+}
+
 // A kernel that allocates tensor memory runs one CTA per SM, so each configuration takes
 // as many pipeline stages as fit in the SM's shared memory.
 template <class F>
@@ -620,13 +1006,19 @@ static auto with_config(int64_t M, F&& f) {
     return f(std::integral_constant<int, 256>{}, std::integral_constant<int, 4>{}, std::false_type{});
 }
 
+// Large M runs on CTA pairs when the device can co-schedule them (the 256 x 256 pair tile).
+static bool use_pairs(int64_t M) { return M > 128 && gemm_pairs() > 0; }
+
+// CTAs whose stream-K flags the GEMM for M rows may use.
 int gemm_ctas(int64_t M) {
+    if (use_pairs(M)) return 2 * gemm_pairs();
     return with_config(M, [](auto bn, auto st, auto sw) -> int {
         return grid_ctas<decltype(bn)::value, decltype(st)::value, decltype(sw)::value>();
     });
 }
 
 size_t gemm_workspace_bytes(int64_t M) {
+    if (use_pairs(M)) return streamk_bytes<256>(2 * gemm_pairs());
     return with_config(M, [](auto bn, auto st, auto sw) -> size_t {
         const int ctas = grid_ctas<decltype(bn)::value, decltype(st)::value, decltype(sw)::value>();
         return ctas < 1 ? 0 : streamk_bytes<decltype(bn)::value>(ctas);
@@ -636,6 +1028,10 @@ size_t gemm_workspace_bytes(int64_t M) {
 // y[M][N] = dec(A) dec(W)^T.  Small M runs swap-AB (weights on the MMA M side).
 int run_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq, const uint8_t* Ws,
                    int64_t N, int64_t K, void* y, int y_fp32, const GemmScratch& ws, cudaStream_t stream, bool pdl) {
+    if (use_pairs(M)) {
+        const GemmOperands op{Aq, As, Wq, Ws, M, N, K, y, N, y_fp32};
+        return launch_gemm_pair(op, ws, gemm_pairs(), stream, pdl);
+    }
     return with_config(M, [&](auto bn, auto st, auto sw) -> int {
         constexpr bool kSwap = decltype(sw)::value;
         const GemmOperands op = kSwap ? GemmOperands{Wq, Ws, Aq, As, N, M, K, y, N, y_fp32}
@@ -644,24 +1040,41 @@ int run_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_
     });
 }
 
-// Layout of the fused linear's workspace: activation codes, their scales, then the GEMM's
-// stream-K scratch (flags first).
+// Layout of the linear's workspace: activation codes, their scales, then the GEMM's stream-K
+// scratch.
 struct LinearWorkspace {
     uint8_t *Aq, *As, *gemm;
     size_t gemm_bytes;
 };
 
+static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
 LinearWorkspace linear_workspace_layout(void* base, int64_t M, int64_t K) {
     LinearWorkspace l;
     l.Aq = static_cast<uint8_t*>(base);
-    l.As = l.Aq + ((M * (K / 2) + 255) / 256) * 256;
-    l.gemm = l.As + ((scale_bytes(M, K) + 255) / 256) * 256;
+    l.As = l.Aq + round256(static_cast<size_t>(M * (K / 2)));
+    l.gemm = l.As + round256(static_cast<size_t>(scale_bytes(M, K)));
     l.gemm_bytes = gemm_workspace_bytes(M);
     return l;
 }
 
 size_t linear_activation_bytes(int64_t M, int64_t K) {
-    return static_cast<size_t>(((M * (K / 2) + 255) / 256) * 256 + ((scale_bytes(M, K) + 255) / 256) * 256);
+    return round256(static_cast<size_t>(M * (K / 2))) + round256(static_cast<size_t>(scale_bytes(M, K)));
+}
+
+// The layer's forward pass on a laid-out workspace: the quantiser (which also clears the
+// GEMM's stream-K flags) and the GEMM, launched with programmatic dependent launch so the
+// GEMM's set-up overlaps the quantiser's tail.  act_mult == nullptr: plain MXFP4 of x (the
+// "pure MXFP4" baseline).  `gemm_scratch`: whether l.gemm holds the stream-K scratch.
+int run_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult, const uint8_t* Wq, const uint8_t* Ws,
+               int64_t N, uint16_t* y, const LinearWorkspace& l, bool gemm_scratch, cudaStream_t st) {
+    uint32_t* flags = gemm_scratch ? reinterpret_cast<uint32_t*>(l.gemm) : nullptr;
+    const int words = gemm_scratch ? gemm_ctas(M) : 0;
+    const int rc = act_mult ? launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, st, flags, words)
+                            : launch_act_quant_plain_clear(x, M, K, l.Aq, l.As, st, flags, words);
+    if (rc) return rc;
+    const GemmScratch ws{gemm_scratch ? l.gemm : nullptr, gemm_scratch ? l.gemm_bytes : 0, false};
+    return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, st, true);
 }
 
 }  // namespace macaq
@@ -703,12 +1116,18 @@ extern "C" int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const 
         !aligned16(workspace))
         return MACAQ_EALIGN;
     if (workspace_bytes < macaq_linear_workspace_bytes(M, N, K)) return MACAQ_EWORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const LinearWorkspace l = linear_workspace_layout(workspace, M, K);
-    // the quantiser also clears the stream-K flags, so the GEMM needs no extra launch
-    if (int rc = launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, st, reinterpret_cast<uint32_t*>(l.gemm),
-                                            gemm_ctas(M)))
-        return rc;
-    const GemmScratch ws{l.gemm, l.gemm_bytes, false};
-    return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, st, true);
+    return run_linear(x, M, K, act_mult, Wq, Ws, N, y, linear_workspace_layout(workspace, M, K), true,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int macaq_mxfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* Wq, const uint8_t* Ws,
+                                  int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!x || !Wq || !Ws || !y || !workspace) return MACAQ_EINVAL;
+    if (int st = check_shape(M, K)) return st;
+    if (int st = check_shape(N, K)) return st;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y) || !aligned16(workspace))
+        return MACAQ_EALIGN;
+    if (workspace_bytes < macaq_linear_workspace_bytes(M, N, K)) return MACAQ_EWORKSPACE;
+    return run_linear(x, M, K, nullptr, Wq, Ws, N, y, linear_workspace_layout(workspace, M, K), true,
+                      static_cast<cudaStream_t>(stream));
 }

@@ -77,12 +77,7 @@ extern "C" int macaq_w4a4_linear_noalloc(const uint16_t* x, int64_t M, int64_t K
     if (act_bytes > kNoAllocScratchBytes) return MACAQ_ETOOLARGE;
     uint8_t* scratch = nullptr;
     if (int st = noalloc_scratch(&scratch)) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const LinearWorkspace l = linear_workspace_layout(scratch, M, K);
     const bool streamk = act_bytes + l.gemm_bytes <= kNoAllocScratchBytes;
-    if (int rc = launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, s, reinterpret_cast<uint32_t*>(l.gemm),
-                                            streamk ? gemm_ctas(M) : 0))
-        return rc;
-    const GemmScratch ws{streamk ? l.gemm : nullptr, streamk ? l.gemm_bytes : 0, false};
-    return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, s, true);
+    return run_linear(x, M, K, act_mult, Wq, Ws, N, y, l, streamk, static_cast<cudaStream_t>(stream));
 }

@@ -32,10 +32,10 @@ enum class QuantMode { kActTransform = 0, kWeightFold = 1, kPlain = 2 };
 
 constexpr int kQuantThreads = 128;
 
-// Eight E2M1 codes of q0..q7 (non-negative) packed two per byte, element 2j in the low
-// nibble: cvt.rn.satfinite.e2m1x2 puts its first source in the high nibble.
-__device__ __forceinline__ uint32_t cvt_e2m1x8(float q0, float q1, float q2, float q3, float q4, float q5,
-                                               float q6, float q7) {
+// Eight E2M1 codes of q0..q7 packed two per byte, element 2j in the low nibble:
+// cvt.rn.satfinite.e2m1x2 puts its first source in the high nibble.  The conversion keeps the
+// IEEE sign, so a negative value that rounds to zero becomes code 0x8 (-0).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 q0, float2 q1, float2 q2, float2 q3) {
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -44,19 +44,24 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float q0, float q1, float q2, flo
         "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
         "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
         : "=r"(out)
-        : "f"(q0), "f"(q1), "f"(q2), "f"(q3), "f"(q4), "f"(q5), "f"(q6), "f"(q7));
+        : "f"(q0.x), "f"(q0.y), "f"(q1.x), "f"(q1.y), "f"(q2.x), "f"(q2.y), "f"(q3.x), "f"(q3.y));
     return out;
 }
 
-// Sign bits of eight values placed on the sign bit (bit 3) of their nibbles.
-__device__ __forceinline__ uint32_t sign_nibbles(const float2* v) {
-    uint32_t s = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        s |= (__float_as_uint(v[j].x) >> 31) << (8 * j + 3);
-        s |= (__float_as_uint(v[j].y) >> 31) << (8 * j + 7);
-    }
-    return s;
+// a - b on both lanes of a float pair, one round-to-nearest rounding each (sm_100 packed op).
+__device__ __forceinline__ float2 fsub2_rn(float2 a, float2 b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+    return *reinterpret_cast<const float2*>(&d);
+}
+
+// max(a, b, c) of three floats (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // 32 raw inputs of one block as 16 pairs (bf16 widened exactly, or fp32).
@@ -114,29 +119,30 @@ __device__ __forceinline__ void scale_fwht32(float2 (&u)[16], const float2 (&m)[
             if ((p & hp) == 0) {
                 const float2 a = u[p], b = u[p + hp];
                 u[p] = __fadd2_rn(a, b);
-                u[p + hp] = __fadd2_rn(a, make_float2(-b.x, -b.y));  // a - b, exactly one rounding
+                u[p + hp] = fsub2_rn(a, b);
             }
         }
     }
 }
 
-// E8M0 scale byte and the 16 code bytes of one transformed block.
+// E8M0 scale byte and the 16 code bytes of one transformed block.  Dividing by the scale
+// 2^(e - 127) is an exact multiplication by 2^(127 - e) (both normal floats).
 __device__ __forceinline__ uint32_t quantize32(const float2 (&v)[16], uint4& codes) {
-    float amax = 0.0f;
+    const float* f = reinterpret_cast<const float*>(v);  // the 32 values in order
+    float amax = fmax3(fabsf(f[0]), fabsf(f[1]), fabsf(f[2]));
 #pragma unroll
-    for (int p = 0; p < 16; ++p) amax = fmaxf(amax, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+    for (int i = 3; i + 1 < 32; i += 2) amax = fmax3(amax, fabsf(f[i]), fabsf(f[i + 1]));
+    amax = fmaxf(amax, fabsf(f[31]));
     const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
     const uint32_t e = E >= 3u ? E - 2u : 0u;
     const float inv = __uint_as_float((254u - e) << 23);  // 2^(127 - e), a normal float
+    const float2 inv2 = make_float2(inv, inv);
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const float2* q = v + 4 * j;
-        w[j] = cvt_e2m1x8(__fmul_rn(fabsf(q[0].x), inv), __fmul_rn(fabsf(q[0].y), inv),
-                          __fmul_rn(fabsf(q[1].x), inv), __fmul_rn(fabsf(q[1].y), inv),
-                          __fmul_rn(fabsf(q[2].x), inv), __fmul_rn(fabsf(q[2].y), inv),
-                          __fmul_rn(fabsf(q[3].x), inv), __fmul_rn(fabsf(q[3].y), inv)) |
-               sign_nibbles(q);
+        w[j] = cvt_e2m1x8(__fmul2_rn(q[0], inv2), __fmul2_rn(q[1], inv2), __fmul2_rn(q[2], inv2),
+                          __fmul2_rn(q[3], inv2));
     }
     codes = make_uint4(w[0], w[1], w[2], w[3]);
     return e;
@@ -234,6 +240,14 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
     const int64_t rpg = quant_rows_per_thread(M, K);
     mx_quant_kernel<QuantMode::kActTransform><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
         x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As, clear, clear_words);
+    return launch_status();
+}
+
+int launch_act_quant_plain_clear(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
+                                 cudaStream_t stream, uint32_t* clear, int clear_words) {
+    const int64_t rpg = quant_rows_per_thread(M, K);
+    mx_quant_kernel<QuantMode::kPlain><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
+        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As, clear, clear_words);
     return launch_status();
 }
 

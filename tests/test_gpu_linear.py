@@ -10,6 +10,7 @@ import torch
 import oracle
 import workloads as wls
 from tests import gpu_util as gu
+from tests import layout
 
 pytestmark = pytest.mark.gpu
 
@@ -75,3 +76,53 @@ def test_linear_workspace_and_errors(mq):
     y2 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N)
     assert torch.equal(y1, y2)
     assert mq.macaq_device_status() == 0
+
+
+# Shapes on both GEMM kernels (swap-AB for M <= 128, the CTA-pair kernel above), with ragged M,
+# N and K tails, padded scale blocks (K = 1056), data-parallel and stream-K schedules.
+LINEAR_SHAPES = [(100, 520, 1024), (129, 520, 1024), (300, 777, 2048), (1000, 1024, 8192), (2049, 2304, 1056),
+                 (4100, 512, 256), (3000, 4096, 768), (2500, 4608, 4352)]
+
+
+@pytest.mark.parametrize("M,N,K", LINEAR_SHAPES, ids=lambda v: str(v))
+def test_linear_matches_two_calls(mq, M, N, K):
+    """The linear reproduces transform-then-GEMM bit for bit, for both the transformed (W4A4)
+    and the plain MXFP4 activations, on a workspace that starts dirty and is reused, and
+    leaves no timeout status."""
+    g = torch.Generator().manual_seed(M + N + K)
+    x = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16).cuda()
+    W = (torch.randn(N, K, generator=g) * 0.05).cuda()
+    s = (torch.rand(K, generator=g) * 3 + 0.3).cuda()
+    Wq, Ws, am = mq.macaq_fold_weights(W, s)
+    Aq, As = mq.macaq_act_transform_quant(x, am)
+    ref = mq.macaq_mxfp4_gemm(Aq, As, Wq, Ws, M, N, K)
+    ws = torch.full((mq.linear_workspace_bytes(M, N, K),), 0x5A, dtype=torch.uint8, device="cuda")
+    y = mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=ws)
+    y2 = mq.macaq_w4a4_linear(x, am, Wq, Ws, N, workspace=ws)  # reused workspace
+    Pq, Ps = mq.macaq_act_quant_plain(x)
+    pref = mq.macaq_mxfp4_gemm(Pq, Ps, Wq, Ws, M, N, K)
+    py = mq.macaq_mxfp4_linear(x, Wq, Ws, N, workspace=ws)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status() == 0
+    assert torch.equal(y, ref)
+    assert torch.equal(y2, ref)
+    assert torch.equal(py, pref)
+    # the workspace starts with the activation codes the linear quantised
+    assert torch.equal(ws[:M * K // 2].view(M, K // 2), Pq)
+
+
+def test_plain_linear_against_oracle(mq):
+    """macaq_mxfp4_linear against the oracle's plain quantiser and fp64 contraction."""
+    M, K, N = 384, 1024, 640
+    g = torch.Generator().manual_seed(77)
+    x = (torch.randn(M, K, generator=g) * 1.5).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g) * 0.03
+    Wq, Ws, _ = mq.macaq_fold_weights(W.cuda(), torch.ones(K, device="cuda"))
+    y = mq.macaq_mxfp4_linear(x.cuda(), Wq, Ws, N)
+    torch.cuda.synchronize()
+    rows = np.arange(0, M, 7)
+    rAq, rAs = oracle.act_quant_plain(x.float().numpy()[rows])
+    Wc = gu.to_np(Wq)
+    Wsr = layout.tiled_to_rowmajor(gu.to_np(Ws), N, K)
+    ref = oracle.mx_gemm(rAq, rAs, Wc, Wsr)
+    assert gu.rel_fro(gu.to_np(y.float())[rows], gu.bf16_round(ref)) <= 1e-3
