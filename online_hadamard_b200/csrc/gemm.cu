@@ -84,7 +84,8 @@ struct GemmParams {
     int y_fp32;
     int num_p_tiles, num_q_tiles, num_k_tiles, q_row_blocks;
     int dp_tiles;         // tiles scheduled data-parallel (blockIdx.x + i * gridDim.x)
-    int64_t sk_units;     // K steps of the remaining tiles, split evenly over the CTAs
+    int64_t sk_units;     // K steps of the remaining tiles, split evenly over the first sk_count units
+    int sk_count;         // scheduling units that take part in the split (<= the units launched)
     float* partials;      // stream-K fp32 partial accumulators, one 128 x BN slot per CTA
     uint32_t* flags;      // stream-K partial-ready counters, one per CTA, zero at launch
     int tma_store;        // bf16 output written by TMA from shared memory (non-swap, N % 8 == 0)
@@ -172,8 +173,8 @@ struct WorkIter {
     // pair kernel (both CTAs of a pair walk the same items).
     __device__ __forceinline__ WorkIter(const GemmParams& p, int id_, int count_) : id(id_), count(count_) {
         dp_next = id;
-        pos = p.sk_units * id / count;
-        hi = p.sk_units * (id + 1) / count;
+        pos = id < p.sk_count ? p.sk_units * id / p.sk_count : 0;
+        hi = id < p.sk_count ? p.sk_units * (id + 1) / p.sk_count : 0;
     }
 
     __device__ __forceinline__ bool next(const GemmParams& p, Work& w) {
@@ -200,7 +201,7 @@ struct WorkIter {
             w.kind = kOwner;
             // last unit whose range holds a K step of this tile: max c with U c / count <= t0 + KT - 1
             const int64_t U = p.sk_units;
-            w.c_last = static_cast<int>(((t0 + KT) * count + U - 1) / U - 1);
+            w.c_last = static_cast<int>(((t0 + KT) * p.sk_count + U - 1) / U - 1);
         } else {
             w.kind = kPartial;
         }
@@ -248,7 +249,7 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
         return;
     }
     if (w.kind == kOwner) {
-        const int64_t U = prm.sk_units, G = e.units;
+        const int64_t U = prm.sk_units, G = prm.sk_count;
         for (int c = e.unit + 1; c <= w.c_last; ++c) {
             if (U * c / G == U * (c + 1) / G) continue;  // empty range: no partial
             const int slot_id = c * e.slot_stride + e.slot_off;
@@ -802,6 +803,39 @@ static int grid_ctas_query() {
 
 // Stream-K scratch of one launch: a flag per CTA (rounded to 256 B) and an fp32 partial
 // accumulator slot (128 x BN) per CTA.
+// Schedule of the persistent grid over `tiles` output tiles of KT K steps on `units`
+// scheduling units (CTAs, or CTA pairs), chosen by its estimated critical path in K steps:
+//   data-parallel  ceil(tiles / units) rounds of whole tiles;
+//   stream-K       all but the last full wave data-parallel, the K steps of the rest split
+//                  evenly over every unit, plus the fix-up's cost `streamk_cost` (needs the
+//                  stream-K scratch).
+// (Splitting only the leftover tiles, each over a few units, measured slower on B200: the
+// owner reads its contributors' partials one after another.)
+struct Schedule {
+    int dp_tiles = 0;
+    int64_t sk_units = 0;
+    int sk_count = 0;
+    int64_t grid = 0;  // units launched
+};
+
+static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch, int streamk_cost) {
+    const int64_t full = tiles / units, rem = tiles % units;
+    const int64_t est_dp = (full + (rem ? 1 : 0)) * KT;
+    const int64_t dp = (full > 0 ? full - 1 : 0) * units;
+    const int64_t est_sk = (dp / units) * KT + ((tiles - dp) * KT + units - 1) / units + streamk_cost;
+    Schedule s;
+    if (scratch && rem != 0 && KT > 1 && est_sk <= est_dp) {
+        s.dp_tiles = static_cast<int>(dp);
+        s.sk_units = (tiles - dp) * static_cast<int64_t>(KT);
+        s.sk_count = static_cast<int>(units);
+        s.grid = units < s.sk_units ? units : s.sk_units;  // every unit gets at least one K step
+    } else {
+        s.dp_tiles = static_cast<int>(tiles);
+        s.grid = units < tiles ? units : tiles;
+    }
+    return s;
+}
+
 template <int BN>
 static size_t streamk_bytes(int ctas) {
     return static_cast<size_t>(((ctas * 4 + 255) / 256) * 256) + static_cast<size_t>(ctas) * kBM * BN * 4;
@@ -828,7 +862,7 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     CUtensorMap mp, mq;
     if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, op.q_rows, op.K, BN))
         return MACAQ_ECUDA;
-    GemmParams prm;
+    GemmParams prm{};
     prm.sf_p = op.ps;
     prm.sf_q = op.qs;
     prm.p_rows = op.p_rows;
@@ -850,30 +884,19 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = mq;  // unused placeholder
     const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
-    int64_t grid = ctas;
-    // Stream-K only with scratch for it, and only where it pays: the data-parallel schedule
-    // runs ceil(tiles / ctas) rounds, stream-K about tiles / ctas rounds plus a fix-up that
-    // costs roughly streamk_cost_steps<BN>() K steps on the critical path (one partial-sum
-    // round trip through L2).
-    const int64_t rounds_dp = (tiles + ctas - 1) / ctas;
-    const int64_t saved_steps = (rounds_dp * ctas - tiles) * prm.num_k_tiles / ctas;
-    const bool streamk = ws.ptr != nullptr && ws.bytes >= streamk_bytes<BN>(ctas) && tiles % ctas != 0 &&
-                         prm.num_k_tiles > 1 && saved_steps >= streamk_cost_steps<BN>();
-    if (streamk) {
-        const int64_t full_waves = tiles / ctas;
-        prm.dp_tiles = static_cast<int>((full_waves > 0 ? full_waves - 1 : 0) * ctas);
-        prm.sk_units = (tiles - prm.dp_tiles) * static_cast<int64_t>(prm.num_k_tiles);
-        if (grid > prm.sk_units) grid = prm.sk_units;  // every CTA gets at least one K step
+    const bool scratch = ws.ptr != nullptr && ws.bytes >= streamk_bytes<BN>(ctas);
+    const Schedule sch = plan_schedule(tiles, ctas, prm.num_k_tiles, scratch, streamk_cost_steps<BN>());
+    const int64_t grid = sch.grid;
+    prm.dp_tiles = sch.dp_tiles;
+    prm.sk_units = sch.sk_units;
+    prm.sk_count = sch.sk_count;
+    prm.flags = nullptr;
+    prm.partials = nullptr;
+    if (sch.sk_units > 0) {
         prm.flags = static_cast<uint32_t*>(ws.ptr);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + ((ctas * 4 + 255) / 256) * 256);
         if (ws.clear_flags && cudaMemsetAsync(prm.flags, 0, sizeof(uint32_t) * ctas, stream) != cudaSuccess)
             return MACAQ_ECUDA;
-    } else {
-        if (grid > tiles) grid = tiles;
-        prm.dp_tiles = static_cast<int>(tiles);
-        prm.sk_units = 0;
-        prm.flags = nullptr;
-        prm.partials = nullptr;
     }
 
     cudaLaunchConfig_t cfg = {};
@@ -934,7 +957,7 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     if (!make_codes_map(&ma, op.pq, op.p_rows, op.K, 128) || !make_codes_map(&mb, op.qq, op.q_rows, op.K, 128) ||
         !make_sf_map(&msa, op.ps, op.p_rows, op.K) || !make_sf_map(&msb, op.qs, op.q_rows, op.K))
         return MACAQ_ECUDA;
-    GemmParams prm;
+    GemmParams prm{};
     prm.sf_p = op.ps;
     prm.sf_q = op.qs;
     prm.p_rows = op.p_rows;
@@ -953,27 +976,20 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     if (!prm.tma_store) my = ma;  // unused placeholder
 
     const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
-    const int64_t rounds_dp = (tiles + pairs - 1) / pairs;
-    const int64_t saved_steps = (rounds_dp * pairs - tiles) * prm.num_k_tiles / pairs;
-    const bool streamk = ws.ptr != nullptr && ws.bytes >= streamk_bytes<256>(2 * pairs) && tiles % pairs != 0 &&
-                         prm.num_k_tiles > 1 && saved_steps >= streamk_cost_steps<256>();
-    int64_t grid_pairs = pairs;
-    if (streamk) {
-        const int64_t full_waves = tiles / pairs;
-        prm.dp_tiles = static_cast<int>((full_waves > 0 ? full_waves - 1 : 0) * pairs);
-        prm.sk_units = (tiles - prm.dp_tiles) * static_cast<int64_t>(prm.num_k_tiles);
-        if (grid_pairs > prm.sk_units) grid_pairs = prm.sk_units;
-        const int ctas = 2 * pairs;
+    const int ctas = 2 * pairs;
+    const bool scratch = ws.ptr != nullptr && ws.bytes >= streamk_bytes<256>(ctas);
+    const Schedule sch = plan_schedule(tiles, pairs, prm.num_k_tiles, scratch, streamk_cost_steps<256>());
+    const int64_t grid_pairs = sch.grid;
+    prm.dp_tiles = sch.dp_tiles;
+    prm.sk_units = sch.sk_units;
+    prm.sk_count = sch.sk_count;
+    prm.flags = nullptr;
+    prm.partials = nullptr;
+    if (sch.sk_units > 0) {
         prm.flags = static_cast<uint32_t*>(ws.ptr);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + ((ctas * 4 + 255) / 256) * 256);
         if (ws.clear_flags && cudaMemsetAsync(prm.flags, 0, sizeof(uint32_t) * ctas, stream) != cudaSuccess)
             return MACAQ_ECUDA;
-    } else {
-        if (grid_pairs > tiles) grid_pairs = tiles;
-        prm.dp_tiles = static_cast<int>(tiles);
-        prm.sk_units = 0;
-        prm.flags = nullptr;
-        prm.partials = nullptr;
     }
 
     cudaLaunchConfig_t cfg = {};
