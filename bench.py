@@ -44,6 +44,21 @@ import workloads as wls  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "W4A4 linear TFLOP/s & % roofline; transform overhead % vs plain MXFP4 GEMM"
+
+
+def linear_roofline(wl, ms, fp4_tflops, hbm_gbs):
+    """The whole linear against its roofline: the slower of its FP4 flops at the tensor peak and
+    its algorithmic bytes (bf16 x, MXFP4 weights, bf16 y, multipliers) at the HBM bandwidth."""
+    t_tensor = wl.flops / (fp4_tflops * 1e12)
+    t_hbm = wls.alg_bytes(wl) / (hbm_gbs * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    return {"bound": "tensor" if t_tensor >= t_hbm else "hbm", "roofline_us": t_roof * 1e6,
+            "achieved_us": ms * 1e3, "frac": t_roof / (ms * 1e-3)}
+
+
+def headline_config(wl, world, l2_note):
+    return {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "parallelism": f"replicas{world}", "l2": l2_note}
 
 
 def load_peaks():
@@ -260,24 +275,26 @@ def time_loop(fn, steps, warmup, device):
 # --------------------------------------------------------------------------- CPU baseline
 
 
-def cpu_baseline(wl, rows=256, max_rows_time=20.0):
-    """The oracle as it stands, on the host cores: transform + quantise `rows` activation
-    rows and contract them with the folded weights (fold excluded: offline)."""
+def cpu_baseline(wl, min_seconds=10.0, max_passes=8):
+    """The oracle as it stands, on the host cores: transform + quantise every activation row
+    and contract them with the folded weights (the fold is offline and excluded), repeated
+    over whole passes of the workload until at least `min_seconds` of CPU work."""
     import oracle
     W = wls.make_w(wl)
     s = wls.make_s(wl, W)
     x = wls.make_x(wl)
     Wq, Ws, a = oracle.fold_weights(W.numpy(), s.numpy())
-    rng = np.random.default_rng(0)
-    idx = np.sort(rng.choice(wl.M, min(rows, wl.M), replace=False))
-    xs = x.float().numpy()[idx]
-    t0 = time.perf_counter()
-    Aq, As = oracle.act_transform_quant(xs, a)
-    oracle.mx_gemm(Aq, As, Wq, Ws)
-    dt = time.perf_counter() - t0
-    flops = 2.0 * len(idx) * wl.N * wl.K
+    xs = x.float().numpy()
+    passes, dt = 0, 0.0
+    while passes < max_passes and (passes == 0 or dt < min_seconds):
+        t0 = time.perf_counter()
+        Aq, As = oracle.act_transform_quant(xs, a)
+        oracle.mx_gemm(Aq, As, Wq, Ws)
+        dt += time.perf_counter() - t0
+        passes += 1
+    flops = passes * wl.flops
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(idx)} of {wl.M} rows of {wl.name} (transform+quant+fp64 GEMM), {dt:.1f} s",
+            "sample": f"{passes} full pass(es) of {wl.name} ({wl.M} rows: transform+quant+fp64 GEMM), {dt:.1f} s",
             "seconds": dt}
 
 
@@ -304,10 +321,11 @@ def run_reference(args):
             times.append(time.perf_counter() - t0)
     dt = sum(times) / len(times)
     val = 2.0 * rows * wl.N * wl.K / dt / 1e12
-    out = {"impl": "reference", "metric": "W4A4 linear TFLOP/s", "value": val, "unit": "TFLOP/s",
+    out = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N},
+           "data": "synthetic",
+           "config": headline_config(wl, int(os.environ.get("WORLD_SIZE", "1")), "oracle on the host cores"),
            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
                             "sample": f"{rows} rows of {wl.M} per step"},
            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -405,16 +423,16 @@ def main():
 
     if rank == 0:
         out = {
-            "metric": "W4A4 linear TFLOP/s (MXFP4 x MXFP4, online scale + FWHT-32 + quant fused ahead of the tcgen05 GEMM)",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4 (e2m1 x e2m1, ue8m0 scales, fp32 accumulate, bf16 out)", "data": "synthetic",
-            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "parallelism": f"replicas{world}",
-                       "l2": f"inputs rotated over {layer.copies} copies (> 3x L2)"},
+            "config": headline_config(wl, world, f"inputs rotated over {layer.copies} copies (> 3x L2)"),
             "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<5> (2-CTA 256x256 tiles)", "achieved": gemm_tflops,
                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
                          "ms_per_launch": ms_gemm},
+            "linear_roofline": linear_roofline(wl, ms, fp4_peak, peaks["hbm_gbs"]),
             "overhead": {"linear_ms": ms, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
                          "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
                          "vs_gemm_only_pct": 100.0 * (ms / ms_gemm - 1.0),
@@ -466,6 +484,8 @@ def secondary(mq, device, peaks, args):
         ms_plain = time_loop(layer.plain, steps, args.warmup, device)
         res[f"{wl.name}_M{M}"] = {"ms": ms, "gbs": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9,
                                    "frac_hbm": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                   "linear_roofline": linear_roofline(wl, ms, peaks["bf16_tflops"] * FP4_OVER_BF16,
+                                                                      peaks["hbm_gbs"]),
                                    "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
         del layer
         torch.cuda.empty_cache()
@@ -476,6 +496,7 @@ def secondary(mq, device, peaks, args):
     ms_gemm = time_loop(layer.gemm, steps, args.warmup, device)
     t = wl.flops / (ms * 1e-3) / 1e12
     res[wl.name] = {"ms": ms, "tflops": t, "frac_fp4_peak": t / (peaks["bf16_tflops"] * FP4_OVER_BF16),
+                    "linear_roofline": linear_roofline(wl, ms, peaks["bf16_tflops"] * FP4_OVER_BF16, peaks["hbm_gbs"]),
                     "gemm_ms": ms_gemm, "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
     del layer
     torch.cuda.empty_cache()
