@@ -91,24 +91,26 @@ def test_gemm_exact_small_integers(mq):
     assert np.array_equal(gu.to_np(y), oracle.mx_gemm(Ac, As, Wc, Ws))
 
 
-def test_gemm_scale_placement(mq):
+@pytest.mark.parametrize("M,N,K", [(128, 256, 512), (512, 512, 1024), (384, 768, 2048)], ids=lambda v: str(v))
+def test_gemm_scale_placement(mq, M, N, K):
     # one distinct scale per (row, block) on both sides: a scale read from the wrong row,
-    # block, TMEM column or byte shows up as a wrong power of two in an isolated product
-    M, N, K = 128, 256, 512
+    # block, TMEM column, lane quadrant or replica shows up as a wrong power of two in an
+    # isolated product.  M <= 128 runs the one-CTA kernel, M > 128 the CTA-pair kernel.
     nb = K // 32
     Ac = np.zeros((M, K // 2), np.uint8)
     Wc = np.zeros((N, K // 2), np.uint8)
-    rng = np.random.default_rng(9)
+    rng = np.random.default_rng(9 + M)
     As = rng.integers(110, 140, (M, nb), dtype=np.uint8)
     Ws = rng.integers(110, 140, (N, nb), dtype=np.uint8)
-    # A row m has a single 1.0 in block m % nb; W row n has a single 1.0 in block n % nb
+    # A row m has a single 1.0 in block m % nb; W row n has a single 1.0 in block (n // 3) % nb
     for m in range(M):
         Ac[m, 16 * (m % nb)] = 0x02
     for n in range(N):
-        Wc[n, 16 * (n % nb)] = 0x02
+        Wc[n, 16 * ((n // 3) % nb)] = 0x02
     y = gu.to_np(mq.macaq_mxfp4_gemm(*to_device_mx(Ac, As, M, K), *to_device_mx(Wc, Ws, N, K), M, N, K,
                                      out_fp32=True))
     ref = oracle.mx_gemm(Ac, As, Wc, Ws)
+    assert np.count_nonzero(ref) > 0
     assert np.array_equal(y, ref)
 
 
