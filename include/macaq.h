@@ -81,8 +81,9 @@ size_t macaq_scale_bytes(int64_t rows, int64_t K);
 int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
 
 /* Bytes of scratch macaq_mxfp4_gemm uses for its stream-K schedule on the current device
- * (a flag and a 128-row fp32 partial-sum slot per CTA of the persistent grid; depends on M
- * and the device's SM count). */
+ * (256 eight-byte flag words and a 128-row fp32 partial-sum slot per CTA of the persistent
+ * grid; depends on M and the device's SM count).  The scratch needs no initialisation: a
+ * flag word counts as written only when it holds the tag of the current launch. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Bytes of scratch macaq_w4a4_linear (and macaq_mxfp4_linear) needs on the current device:
@@ -150,7 +151,9 @@ int macaq_w4a4_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_
  *   macaq_gemm_workspace_bytes(M, N, K) the GEMM balances its last wave with a stream-K
  *   split of the K steps (partial sums added in a fixed order, so results are
  *   deterministic); with workspace = NULL it runs a data-parallel schedule.  Both
- *   schedules accumulate in fp32 and agree within fp32 summation order.
+ *   schedules accumulate in fp32 and agree within fp32 summation order.  The workspace's
+ *   contents on entry and on return are unspecified; calls sharing one workspace must be
+ *   stream-ordered.
  */
 int macaq_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                           void* stream);

@@ -29,6 +29,8 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <mutex>
 #include <type_traits>
@@ -39,9 +41,9 @@
 namespace macaq {
 
 int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
-                               uint8_t* Aq, uint8_t* As, cudaStream_t stream, uint32_t* clear, int clear_words);
-int launch_act_quant_plain_clear(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
-                                 cudaStream_t stream, uint32_t* clear, int clear_words);
+                               uint8_t* Aq, uint8_t* As, cudaStream_t stream);
+int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
+                           cudaStream_t stream);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -87,7 +89,8 @@ struct GemmParams {
     int64_t sk_units;     // K steps of the remaining tiles, split evenly over the first sk_count units
     int sk_count;         // scheduling units that take part in the split (<= the units launched)
     float* partials;      // stream-K fp32 partial accumulators, one 128 x BN slot per CTA
-    uint32_t* flags;      // stream-K partial-ready counters, one per CTA, zero at launch
+    uint64_t* flags;      // stream-K hand-off: one word per (partial slot, epilogue thread)
+    uint64_t tag;         // this launch's value of a written flag word (unique per launch)
     int tma_store;        // bf16 output written by TMA from shared memory (non-swap, N % 8 == 0)
 };
 
@@ -210,6 +213,16 @@ struct WorkIter {
     }
 };
 
+__device__ __forceinline__ uint64_t ld_acquire64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -236,16 +249,17 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
     constexpr int kHalf = BN / 2;
     constexpr int kChunk = kHalf >= 32 ? 32 : kHalf;
     if (w.kind == kPartial) {
-        // fp32 partial to this CTA's slot, [chunk of 4 columns][epilogue thread]; the slot's
-        // counter reaches kEpiThreads once every thread's part is visible
+        // fp32 partial to this CTA's slot, [chunk of 4 columns][epilogue thread]; then this
+        // thread's flag word takes the launch's tag (release: after its part of the partial).
+        // The owner's thread with the same index reads exactly this part, so no flag is
+        // ever shared, counted or cleared.
         float4* slot = reinterpret_cast<float4*>(prm.partials + static_cast<int64_t>(e.slot_self) * (kBM * BN));
 #pragma unroll
         for (int j = 0; j < kHalf / 4; ++j)
             __stcg(slot + j * kEpiThreads + e.etid,
                    make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
-        __threadfence();
-        atomicAdd(prm.flags + e.slot_self, 1u);
+        st_release(prm.flags + static_cast<int64_t>(e.slot_self) * kEpiThreads + e.etid, prm.tag);
         return;
     }
     if (w.kind == kOwner) {
@@ -255,7 +269,8 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
             const int slot_id = c * e.slot_stride + e.slot_off;
             if (!abort) {
                 const long long t0 = clock64();
-                while (ld_acquire(prm.flags + slot_id) < static_cast<uint32_t>(kEpiThreads)) {
+                const uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + e.etid;
+                while (ld_acquire64(flag) != prm.tag) {
                     if (clock64() - t0 > kWaitLimitCycles) {
                         atomicExch(&g_device_status, MACAQ_ETIMEOUT);
                         abort = 1;
@@ -448,7 +463,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t acc_phase = 0;
         WorkIter it(prm, blockIdx.x, gridDim.x);
         Work w;
-        if (prm.sk_units > 0) griddep_wait();  // the flags were cleared by the kernel launched before
         while (!abort && it.next(prm, w)) {
             const int pt = w.tile % prm.num_p_tiles;
             const int qt = w.tile / prm.num_p_tiles;
@@ -656,7 +670,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t acc_phase = 0;
         WorkIter it(prm, pair, pairs);
         Work w;
-        if (prm.sk_units > 0) griddep_wait();
         while (!abort && it.next(prm, w)) {
             const int pt = w.tile / prm.num_q_tiles;  // activation-block major: early tiles need early rows
             const int qt = w.tile % prm.num_q_tiles;
@@ -836,9 +849,26 @@ static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch
     return s;
 }
 
+// Stream-K scratch: a flag word per (CTA slot, epilogue thread), then one 128 x BN fp32
+// partial-sum slot per CTA.  Flags hold the tag of the launch that last wrote them, so the
+// scratch needs no clearing: any contents on entry are fine.
+static size_t streamk_flag_bytes(int ctas) {
+    return (static_cast<size_t>(ctas) * kEpiThreads * 8 + 255) / 256 * 256;
+}
+
 template <int BN>
 static size_t streamk_bytes(int ctas) {
-    return static_cast<size_t>(((ctas * 4 + 255) / 256) * 256) + static_cast<size_t>(ctas) * kBM * BN * 4;
+    return streamk_flag_bytes(ctas) + static_cast<size_t>(ctas) * kBM * BN * 4;
+}
+
+// A value no flag word of any earlier launch in this process holds: a per-process random
+// start, then one step per launch.
+static uint64_t next_launch_tag() {
+    static std::atomic<uint64_t> next{[] {
+        const uint64_t t = static_cast<uint64_t>(std::chrono::high_resolution_clock::now().time_since_epoch().count());
+        return (t * 0x9E3779B97F4A7C15ull) | 1ull;
+    }()};
+    return next.fetch_add(2, std::memory_order_relaxed);
 }
 
 struct GemmOperands {
@@ -849,11 +879,10 @@ struct GemmOperands {
     int y_fp32;
 };
 
-// Scratch of the stream-K schedule and where its flags must be cleared before the GEMM.
+// Scratch of the stream-K schedule (nullptr: data-parallel schedule only).
 struct GemmScratch {
-    void* ptr;            // nullptr: data-parallel schedule only
+    void* ptr;
     size_t bytes;
-    bool clear_flags;     // clear the flags here (false: an earlier kernel on the stream did)
 };
 
 template <int BN, int STAGES, bool SWAP>
@@ -893,10 +922,9 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     prm.flags = nullptr;
     prm.partials = nullptr;
     if (sch.sk_units > 0) {
-        prm.flags = static_cast<uint32_t*>(ws.ptr);
-        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + ((ctas * 4 + 255) / 256) * 256);
-        if (ws.clear_flags && cudaMemsetAsync(prm.flags, 0, sizeof(uint32_t) * ctas, stream) != cudaSuccess)
-            return MACAQ_ECUDA;
+        prm.flags = static_cast<uint64_t*>(ws.ptr);
+        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + streamk_flag_bytes(ctas));
+        prm.tag = next_launch_tag();
     }
 
     cudaLaunchConfig_t cfg = {};
@@ -986,10 +1014,9 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     prm.flags = nullptr;
     prm.partials = nullptr;
     if (sch.sk_units > 0) {
-        prm.flags = static_cast<uint32_t*>(ws.ptr);
-        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + ((ctas * 4 + 255) / 256) * 256);
-        if (ws.clear_flags && cudaMemsetAsync(prm.flags, 0, sizeof(uint32_t) * ctas, stream) != cudaSuccess)
-            return MACAQ_ECUDA;
+        prm.flags = static_cast<uint64_t*>(ws.ptr);
+        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + streamk_flag_bytes(ctas));
+        prm.tag = next_launch_tag();
     }
 
     cudaLaunchConfig_t cfg = {};
@@ -1078,18 +1105,16 @@ size_t linear_activation_bytes(int64_t M, int64_t K) {
     return round256(static_cast<size_t>(M * (K / 2))) + round256(static_cast<size_t>(scale_bytes(M, K)));
 }
 
-// The layer's forward pass on a laid-out workspace: the quantiser (which also clears the
-// GEMM's stream-K flags) and the GEMM, launched with programmatic dependent launch so the
-// GEMM's set-up overlaps the quantiser's tail.  act_mult == nullptr: plain MXFP4 of x (the
-// "pure MXFP4" baseline).  `gemm_scratch`: whether l.gemm holds the stream-K scratch.
+// The layer's forward pass on a laid-out workspace: the quantiser, then the GEMM launched with
+// programmatic dependent launch so its set-up overlaps the quantiser's tail.  act_mult ==
+// nullptr: plain MXFP4 of x (the "pure MXFP4" baseline).  `gemm_scratch`: whether l.gemm
+// holds the stream-K scratch.
 int run_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult, const uint8_t* Wq, const uint8_t* Ws,
                int64_t N, uint16_t* y, const LinearWorkspace& l, bool gemm_scratch, cudaStream_t st) {
-    uint32_t* flags = gemm_scratch ? reinterpret_cast<uint32_t*>(l.gemm) : nullptr;
-    const int words = gemm_scratch ? gemm_ctas(M) : 0;
-    const int rc = act_mult ? launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, st, flags, words)
-                            : launch_act_quant_plain_clear(x, M, K, l.Aq, l.As, st, flags, words);
+    const int rc = act_mult ? launch_act_transform_quant(x, M, K, act_mult, l.Aq, l.As, st)
+                            : launch_act_quant_plain(x, M, K, l.Aq, l.As, st);
     if (rc) return rc;
-    const GemmScratch ws{gemm_scratch ? l.gemm : nullptr, gemm_scratch ? l.gemm_bytes : 0, false};
+    const GemmScratch ws{gemm_scratch ? l.gemm : nullptr, gemm_scratch ? l.gemm_bytes : 0};
     return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, st, true);
 }
 
@@ -1118,7 +1143,7 @@ extern "C" int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M,
         (workspace && !aligned16(workspace)))
         return MACAQ_EALIGN;
     if (workspace && workspace_bytes < gemm_workspace_bytes(M)) return MACAQ_EWORKSPACE;
-    const GemmScratch ws{workspace, workspace ? workspace_bytes : 0, true};
+    const GemmScratch ws{workspace, workspace ? workspace_bytes : 0};
     return run_mxfp4_gemm(Aq, As, M, Wq, Ws, N, K, y, y_is_fp32, ws, static_cast<cudaStream_t>(stream), false);
 }
 

@@ -166,10 +166,8 @@ template <QuantMode MODE>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
     const void* __restrict__ in, int64_t R, int64_t K, int64_t rpg, const float* __restrict__ mult,
     const float* __restrict__ s, double c, float* __restrict__ act_mult_out, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, uint32_t* __restrict__ clear, int clear_words) {
+    uint8_t* __restrict__ scales) {
     griddep_launch_dependents();
-    if (blockIdx.x == 0)  // words the next kernel on the stream needs zeroed (GEMM stream-K flags)
-        for (int i = threadIdx.x; i < clear_words; i += kQuantThreads) clear[i] = 0u;
     const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
@@ -233,21 +231,12 @@ static unsigned quant_blocks(int64_t R, int64_t K, int64_t rpg) {
     return static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
 }
 
-// Launch helpers used by the C entry points and by the fused linear.
+// Launch helpers used by the C entry points and by the linear.
 int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
-                               uint8_t* Aq, uint8_t* As, cudaStream_t stream, uint32_t* clear = nullptr,
-                               int clear_words = 0) {
+                               uint8_t* Aq, uint8_t* As, cudaStream_t stream) {
     const int64_t rpg = quant_rows_per_thread(M, K);
     mx_quant_kernel<QuantMode::kActTransform><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
-        x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As, clear, clear_words);
-    return launch_status();
-}
-
-int launch_act_quant_plain_clear(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
-                                 cudaStream_t stream, uint32_t* clear, int clear_words) {
-    const int64_t rpg = quant_rows_per_thread(M, K);
-    mx_quant_kernel<QuantMode::kPlain><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
-        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As, clear, clear_words);
+        x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As);
     return launch_status();
 }
 
@@ -255,7 +244,7 @@ int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq,
                            cudaStream_t stream) {
     const int64_t rpg = quant_rows_per_thread(M, K);
     mx_quant_kernel<QuantMode::kPlain><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
-        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As, nullptr, 0);
+        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As);
     return launch_status();
 }
 
@@ -297,6 +286,6 @@ extern "C" int macaq_fold_weights(const float* W, int64_t N, int64_t K, const fl
     const double c = 1.0 / std::sqrt(32.0);  // correctly rounded (IEEE sqrt and divide)
     const int64_t rpg = quant_rows_per_thread(N, K);
     mx_quant_kernel<QuantMode::kWeightFold><<<quant_blocks(N, K, rpg), kQuantThreads, 0, st>>>(
-        W, N, K, rpg, nullptr, s, c, act_mult, Wq, Ws, nullptr, 0);
+        W, N, K, rpg, nullptr, s, c, act_mult, Wq, Ws);
     return launch_status();
 }

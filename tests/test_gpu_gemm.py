@@ -78,6 +78,26 @@ def test_gemm_identical_codes(mq, M, N, K):
     assert np.max(np.abs(gu.to_np(y32) - ref)) <= 1e-3 * np.max(np.abs(ref)) + 1e-30
 
 
+# both shapes take the stream-K schedule (one-CTA swap-AB and CTA-pair kernels)
+@pytest.mark.parametrize("M,N,K", [(16, 2048, 8192), (300, 2048, 16384)], ids=lambda v: str(v))
+def test_streamk_workspace_reused_and_dirty(mq, M, N, K):
+    """Stream-K hand-off through a workspace that is reused call after call and starts with
+    arbitrary bytes (flag words only count when they hold the current launch's tag): five
+    calls in a row, each bit-identical to the first."""
+    rng = np.random.default_rng(M + K)
+    Ac, As = random_mx(rng, M, K)
+    Wc, Ws = random_mx(rng, N, K)
+    Ag, Asg = to_device_mx(Ac, As, M, K)
+    Wg, Wsg = to_device_mx(Wc, Ws, N, K)
+    ws = torch.randint(0, 256, (mq.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    ys = [mq.macaq_mxfp4_gemm(Ag, Asg, Wg, Wsg, M, N, K, out_fp32=True, workspace=ws) for _ in range(5)]
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status() == 0
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+    assert gu.rel_fro(gu.to_np(ys[0]), oracle.mx_gemm(Ac, As, Wc, Ws)) <= TOL
+
+
 def test_gemm_exact_small_integers(mq):
     # all elements in {0, +-0.5, +-1} and scale 127: every partial sum is exact in fp32
     rng = np.random.default_rng(5)
