@@ -47,6 +47,55 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "W4A4 linear TFLOP/s & % roofline; transform overhead % vs plain MXFP4 GEMM"
 
 
+class Ranks:
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE), replicas of the layer:
+    the process group serves only the barriers around the timed region and the max over ranks
+    of the device time (no data-path collective).  `backend` is "nccl" on GPUs; tests use
+    "gloo" on the CPU."""
+
+    def __init__(self, world, rank, local, backend):
+        self.world, self.rank, self.local = world, rank, local
+        self.dist = None
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            self.device = torch.device("cuda", local)
+        else:
+            self.device = torch.device("cpu")
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.dist = dist
+
+    @classmethod
+    def from_env(cls, backend):
+        return cls(int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                   int(os.environ.get("LOCAL_RANK", "0")), backend)
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v):
+        """The largest of every rank's v (every rank gets it)."""
+        if self.dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def whole_job_tflops(world, flops_per_rank, ms_max):
+    """Throughput of the whole job: every rank's work over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def linear_roofline(wl, ms, fp4_tflops, hbm_gbs):
     """The whole linear against its roofline: the slower of its FP4 flops at the tensor peak and
     its algorithmic bytes (bf16 x, MXFP4 weights, bf16 y, multipliers) at the HBM bandwidth."""
@@ -356,17 +405,9 @@ def main():
         run_reference(args)
         return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
+    ranks = Ranks.from_env("nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
+    device = ranks.device
 
     import online_hadamard_b200 as mq
     mq.load_library()
@@ -376,16 +417,8 @@ def main():
     wl = wls.LLAMA_UP
     layer = Layer(mq, wl, device)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = ranks.barrier
+    max_over_ranks = ranks.max
 
     # ---- headline: the fused linear, K steps captured in one CUDA graph
     loop = GraphLoop(layer.linear, args.steps, args.warmup, device)
@@ -401,7 +434,7 @@ def main():
     clk = clocks.stop()
     del loop
     ms = max_over_ranks(ms_total / args.steps)
-    value = world * wl.flops / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, wl.flops, ms)
 
     # ---- dominant kernel, the comparators and end to end (same rotation)
     ms_gemm = time_loop(layer.gemm, args.steps, args.warmup, device)
@@ -438,7 +471,7 @@ def main():
                          "vs_gemm_only_pct": 100.0 * (ms / ms_gemm - 1.0),
                          "transform_quant_ms": ms_xform,
                          "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
-            "e2e": {"value": world * wl.flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+            "e2e": {"value": whole_job_tflops(world, wl.flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": wl.M * wl.K * 2, "d2h_bytes_per_step": wl.M * wl.N * 2},
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
@@ -447,8 +480,7 @@ def main():
             "secondary": extra,
         }
         print(json.dumps(out))
-    if dist is not None:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def profile_kernels(name):
