@@ -68,6 +68,7 @@ def _load():
             lib.oracle_fold_weights.argtypes = [p, i64, i64, p, p, p, p]
             lib.oracle_mx_decode.argtypes = [p, p, i64, i64, p]
             lib.oracle_mx_gemm.argtypes = [p, p, p, i64, p, p, i64, i64, p]
+            lib.oracle_calibrate_scale.argtypes = [p, i64, p, i64, i64, p]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -200,6 +201,20 @@ def mx_gemm(Aq, As, Wq, Ws, rows=None) -> np.ndarray:
     _load().oracle_mx_gemm(_ptr(Aq), _ptr(As), None if rows_arr is None else _ptr(rows_arr), n_rows,
                            _ptr(Wq), _ptr(Ws), N, K, _ptr(y))
     return y
+
+
+def calibrate_scale(xcal, W) -> np.ndarray:
+    """Per-channel scale s [K] from calibration activations xcal [C, K] and weights W [N, K]:
+    fl32(sqrt(max|xcal_:,j| / max|W_:,j|)) in double, 1 where either maximum is 0."""
+    xcal = _f32(xcal)
+    W = _f32(W)
+    C, K = xcal.shape
+    N, K2 = W.shape
+    if K2 != K:
+        raise ValueError("xcal and W must have the same K")
+    s = np.empty(K, np.float32)
+    _load().oracle_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s))
+    return s
 
 
 def num_threads() -> int:

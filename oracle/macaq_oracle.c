@@ -34,6 +34,11 @@
  *
  * The GEMM is the exact contraction of decoded values in fp64.
  *
+ * Calibration of s (the step before the fold; the pages name calibration but give no rule):
+ * s_j = fl32(sqrt(max_r |xcal_rj| / max_n |W_nj|)) with the maxima, the quotient and the root
+ * in IEEE double -- the SmoothQuant alpha = 1/2 balance, after which max|x_j / s_j| and
+ * max|W_nj * s_j| agree; s_j = 1 when either maximum is zero (nothing to balance).
+ *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fPIC -shared (no -ffast-math, no -march):
  * every fp32 operation above must be one IEEE round-to-nearest operation.
  */
@@ -236,6 +241,18 @@ void oracle_mx_gemm(const uint8_t* Aq, const uint8_t* As, const int64_t* rows, i
 }
 
 /* Number of OpenMP threads the oracle runs with (reported beside its timings). */
+/* Per-channel scale from a calibration batch xcal [C][K] (bf16 values held in fp32) and the
+ * weights W [N][K]: column maxima of |.|, then sqrt of their quotient in double, rounded once to
+ * fp32; 1 for a column whose activation or weight maximum is zero. */
+void oracle_calibrate_scale(const float* xcal, int64_t C, const float* W, int64_t N, int64_t K, float* s) {
+    for (int64_t j = 0; j < K; ++j) {
+        double ax = 0.0, aw = 0.0;
+        for (int64_t r = 0; r < C; ++r) ax = fmax(ax, fabs((double)xcal[r * K + j]));
+        for (int64_t n = 0; n < N; ++n) aw = fmax(aw, fabs((double)W[n * K + j]));
+        s[j] = (ax == 0.0 || aw == 0.0) ? 1.0f : (float)sqrt(ax / aw);
+    }
+}
+
 int oracle_num_threads(void) {
     int n = 1;
 #pragma omp parallel

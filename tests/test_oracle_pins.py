@@ -415,3 +415,41 @@ def test_end_to_end_quantisation_error_is_reported():
     rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert rel < 0.5  # W4A4 on a 256-wide dot product: a few percent is typical
     print(f"tiny: W4A4 relative Frobenius error vs fp64 x W^T = {rel:.4f}")
+
+
+# ---- calibration of the per-channel scale (the step before the fold) ----
+
+def test_calibrate_scale_hand_values():
+    # column maxima (ignoring sign) 4/1, 1/4, 9/1, 3/3, and zero columns -> 1
+    xcal = np.array([[4.0, -1.0, 9.0, 3.0, 0.0, 2.0],
+                     [-2.0, 0.5, 1.0, -3.0, 0.0, 1.0]], np.float32)
+    W = np.array([[1.0, 4.0, -1.0, 3.0, 5.0, 0.0],
+                  [-0.5, -2.0, 0.25, 1.0, 1.0, 0.0]], np.float32)
+    s = oracle.calibrate_scale(xcal, W)
+    assert s.tolist() == [2.0, 0.5, 3.0, 1.0, 1.0, 1.0]
+
+
+def test_calibrate_scale_power_of_two_and_sign_invariance():
+    rng = np.random.default_rng(3)
+    xcal = (rng.standard_normal((64, 96)) * 3).astype(np.float32)
+    W = (rng.standard_normal((40, 96)) * 0.02).astype(np.float32)
+    s = oracle.calibrate_scale(xcal, W)
+    # W x 4 halves s exactly, x x 4 doubles it; signs do not matter
+    assert np.array_equal(oracle.calibrate_scale(xcal, W * 4), s / 2)
+    assert np.array_equal(oracle.calibrate_scale(xcal * 4, W), s * 2)
+    assert np.array_equal(oracle.calibrate_scale(-xcal, -W), s)
+    # permuting channels permutes s
+    perm = rng.permutation(96)
+    assert np.array_equal(oracle.calibrate_scale(xcal[:, perm], W[:, perm]), s[perm])
+
+
+def test_calibrate_scale_balances_activation_and_weight_ranges():
+    # the purpose of the rule: after scaling, each channel's activation range max|x/s| and
+    # weight range max|W s| coincide (up to rounding s to fp32)
+    rng = np.random.default_rng(4)
+    xcal = (rng.standard_normal((64, 128)) * rng.uniform(0.1, 50, 128)).astype(np.float32)
+    W = (rng.standard_normal((200, 128)) * rng.uniform(0.001, 0.1, 128)).astype(np.float32)
+    s = oracle.calibrate_scale(xcal, W).astype(np.float64)
+    xr = np.abs(xcal.astype(np.float64)).max(0) / s
+    wr = np.abs(W.astype(np.float64)).max(0) * s
+    np.testing.assert_allclose(xr, wr, rtol=2.0 ** -22)
