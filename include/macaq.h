@@ -92,6 +92,21 @@ size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 size_t macaq_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
+ * macaq_calibrate_scale -- the per-channel scale s before the fold (Abstract: the method is
+ * calibrated per layer; the pages give no rule).  The rule used is the SmoothQuant 1/2
+ * balance: s_j = fl32(sqrt(max_r |xcal_rj| / max_n |W_nj|)), quotient and root in IEEE double
+ * (correctly rounded), s_j = 1 where either maximum is 0; afterwards max|x_j / s_j| and
+ * max|W_nj * s_j| agree.
+ *   xcal  in   bf16 bit patterns [C][K], a calibration batch of activations
+ *   W     in   fp32 [N][K]
+ *   s     out  fp32 [K]; usable by macaq_fold_weights as is
+ * Offline, asynchronous on `stream` (a memset and two kernels; reads W once).  NaN or infinite
+ * inputs give undefined s.  MACAQ_ESHAPE for K % 32 != 0, C or N out of range.
+ */
+int macaq_calibrate_scale(const uint16_t* xcal, int64_t C, const float* W, int64_t N, int64_t K,
+                          float* s, void* stream);
+
+/*
  * macaq_fold_weights -- offline weight preparation (Abstract: "absorbing the corresponding
  * inverse transforms into its weights"; weights quantised round-to-nearest).
  *   W        in   fp32 [N][K]

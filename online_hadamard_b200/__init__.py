@@ -23,7 +23,7 @@ from . import build as _build_mod
 
 __all__ = [
     "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes", "gemm_workspace_bytes",
-    "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
+    "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_linear_noalloc",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
@@ -32,7 +32,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "macaq_status_str", "macaq_scale_bytes", "macaq_scale_offset", "macaq_linear_workspace_bytes",
     "macaq_gemm_workspace_bytes",
-    "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
+    "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
     "macaq_act_quant_plain", "macaq_mxfp4_linear", "macaq_mxfp4_gemm", "macaq_device_status",
     "macaq_w4a4_linear_noalloc",
 )
@@ -70,6 +70,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_linear_workspace_bytes.restype = sz
         lib.macaq_gemm_workspace_bytes.argtypes = [i64, i64, i64]
         lib.macaq_gemm_workspace_bytes.restype = sz
+        lib.macaq_calibrate_scale.argtypes = [p, i64, p, i64, i64, p, p]
         lib.macaq_fold_weights.argtypes = [p, i64, i64, p, p, p, p, p]
         lib.macaq_act_transform_quant.argtypes = [p, i64, i64, p, p, p, p]
         lib.macaq_act_quant_plain.argtypes = [p, i64, i64, p, p, p]
@@ -78,7 +79,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_mxfp4_linear.argtypes = [p, i64, i64, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
         lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
-        for name in ("macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
+        for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_linear_noalloc"):
             getattr(lib, name).restype = i32
@@ -134,6 +135,21 @@ def linear_workspace_bytes(M: int, N: int, K: int) -> int:
 def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     """Scratch bytes of the GEMM's stream-K schedule on the current device."""
     return int(load_library().macaq_gemm_workspace_bytes(M, N, K))
+
+
+def macaq_calibrate_scale(xcal: torch.Tensor, W: torch.Tensor, s=None, stream=None):
+    """Per-channel scale s (fp32 [K]) from a bf16 calibration batch [C, K] and fp32 weights [N, K]."""
+    C, K = xcal.shape
+    _need(xcal, "xcal", torch.bfloat16)
+    _need(W, "W", torch.float32)
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("xcal and W must have the same K")
+    s = torch.empty(K, dtype=torch.float32, device=W.device) if s is None else s
+    _need(s, "s", torch.float32, (K,))
+    _check(load_library().macaq_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s), _stream(stream)),
+           "macaq_calibrate_scale")
+    return s
 
 
 def macaq_fold_weights(W: torch.Tensor, s: torch.Tensor, Wq=None, Ws=None, act_mult=None, stream=None):

@@ -87,3 +87,13 @@ def test_validation_null_shape_alignment():
                  None) == -3
     # bad flag
     assert _call("macaq_mxfp4_gemm", P(FAKE), P(FAKE), 4, P(FAKE), P(FAKE), 8, 64, P(FAKE), 2, None, 0, None) == -1
+
+
+def test_calibrate_scale_validation():
+    P = ctypes.c_void_p
+    assert _call("macaq_calibrate_scale", None, 64, P(FAKE), 128, 256, P(FAKE), None) == -1
+    assert _call("macaq_calibrate_scale", P(FAKE), 64, P(FAKE), 128, 256, None, None) == -1
+    assert _call("macaq_calibrate_scale", P(FAKE), 0, P(FAKE), 128, 256, P(FAKE), None) == -2
+    assert _call("macaq_calibrate_scale", P(FAKE), 64, P(FAKE), 0, 256, P(FAKE), None) == -2
+    assert _call("macaq_calibrate_scale", P(FAKE), 64, P(FAKE), 128, 200, P(FAKE), None) == -2
+    assert _call("macaq_calibrate_scale", P(FAKE), 64, P(MIS), 128, 256, P(FAKE), None) == -3

@@ -145,11 +145,16 @@ def make_w(w: Workload) -> torch.Tensor:
     return torch.randn(w.N, w.K, generator=g, dtype=torch.float32) * w.w_std
 
 
+def make_xcal(w: Workload) -> torch.Tensor:
+    """The separate 64-token bf16 calibration batch of a workload (same distribution as x)."""
+    return _draw_x(w, CALIB_TOKENS, 2).to(torch.bfloat16)
+
+
 def make_s(w: Workload, W: torch.Tensor | None = None) -> torch.Tensor:
     """Per-channel scale s (fp32 [K], > 0) from a separate 64-token calibration batch."""
     if W is None:
         W = make_w(w)
-    xcal = _draw_x(w, CALIB_TOKENS, 2).to(torch.bfloat16).to(torch.float64)
+    xcal = make_xcal(w).to(torch.float64)
     xmax = xcal.abs().amax(0)
     wmax = W.to(torch.float64).abs().amax(0)
     s = torch.sqrt(xmax / wmax)
