@@ -392,6 +392,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 64-layer stack sweep")
     ap.add_argument("--profile", default=None, metavar="WORKLOAD",
                     help="run each kernel of one workload three times (for ncu captures) and exit; "
                          "WORKLOAD is a name from workloads.py, optionally with _M<m>")
@@ -449,6 +450,8 @@ def main():
     extra = {}
     if not args.no_extra:
         extra = secondary(mq, device, peaks, args)
+    if not args.no_stack:
+        extra["qwen3_32b_stack"] = stack_sweep(mq, device, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -503,6 +506,54 @@ def profile_kernels(name):
         mq.macaq_mxfp4_gemm(Aq, As, Wq, Ws, wl.M, wl.N, wl.K, y=y, workspace=gws)
     torch.cuda.synchronize()
     print(f"profiled {wl.name} M={wl.M} K={wl.K} N={wl.N}")
+
+
+def stack_sweep(mq, device, peaks, Ms=(1, 32, 512, 4096), steps=3, warmup=2):
+    """The 64-layer Qwen3-32B-shaped linear stack (q, k, v, o, gate, up, down per layer): each
+    linear's weights and calibration batch are drawn on the device, s is calibrated and W folded
+    by the library, and the fp32 weights are freed before the next linear, so only the 16.6 GB
+    of MXFP4 weights stay resident.  Per M, all 448 linears run back to back in one CUDA graph,
+    as W4A4 linears and as plain-MXFP4 linears; the summed times give the transform's overhead."""
+    lin = []
+    for layer in range(64):
+        for name, K, N in wls.QWEN_STACK_LINEARS:
+            wl = wls.stack_layer(layer, name, 1)
+            W = wls.make_w_device(wl, device)
+            s = mq.macaq_calibrate_scale(wls.make_x_device(wl, wls.CALIB_TOKENS, device, tensor_id=2), W)
+            Wq, Ws, am = mq.macaq_fold_weights(W, s)
+            del W
+            lin.append((K, N, Wq, Ws, am))
+    torch.cuda.empty_cache()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    res = {"layers": 64, "linears": len(lin), "weights_gb": sum(q.numel() + t.numel() for _, _, q, t, _ in lin) / 1e9}
+    for M in Ms:
+        xs = {K: wls.make_x_device(wls.stack_layer(0, name, M), M, device)
+              for name, K, _ in wls.QWEN_STACK_LINEARS}
+        ys = {N: torch.empty(M, N, dtype=torch.bfloat16, device=device) for _, _, N in wls.QWEN_STACK_LINEARS}
+        ws = torch.empty(max(mq.linear_workspace_bytes(M, N, K) for _, K, N in wls.QWEN_STACK_LINEARS),
+                         dtype=torch.uint8, device=device)
+
+        def w4a4(i):
+            for K, N, Wq, Ws, am in lin:
+                mq.macaq_w4a4_linear(xs[K], am, Wq, Ws, N, y=ys[N], workspace=ws)
+
+        def plain(i):
+            for K, N, Wq, Ws, am in lin:
+                mq.macaq_mxfp4_linear(xs[K], Wq, Ws, N, y=ys[N], workspace=ws)
+
+        ms = time_loop(w4a4, steps, warmup, device)
+        ms_plain = time_loop(plain, steps, warmup, device)
+        flops = sum(2.0 * M * K * N for K, N, *_ in lin)
+        nbytes = sum(wls.alg_bytes(wls.Workload("", 5, M, K, N, "normal", 0.0, 1.0)) for K, N, *_ in lin)
+        t_roof = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+        res[f"M{M}"] = {"w4a4_ms": ms, "plain_mxfp4_ms": ms_plain, "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
+                        "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                        "linear_roofline_frac": t_roof / (ms * 1e-3)}
+        del xs, ys, ws
+        torch.cuda.empty_cache()
+    del lin
+    torch.cuda.empty_cache()
+    return res
 
 
 def secondary(mq, device, peaks, args):

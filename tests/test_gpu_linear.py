@@ -80,7 +80,7 @@ def test_linear_workspace_and_errors(mq):
 
 # Shapes on both GEMM kernels (swap-AB for M <= 128, the CTA-pair kernel above), with ragged M,
 # N and K tails, padded scale blocks (K = 1056), data-parallel and stream-K schedules.
-LINEAR_SHAPES = [(1, 384, 256), (33, 2048, 8192), (128, 1000, 1056), (100, 520, 1024), (129, 520, 1024), (300, 777, 2048), (1000, 1024, 8192), (2049, 2304, 1056),
+LINEAR_SHAPES = [(1, 384, 256), (8, 512, 8192), (16, 1000, 6144), (3, 2000, 5120), (33, 2048, 8192), (128, 1000, 1056), (100, 520, 1024), (129, 520, 1024), (300, 777, 2048), (1000, 1024, 8192), (2049, 2304, 1056),
                  (4100, 512, 256), (3000, 4096, 768), (2500, 4608, 4352)]
 
 

@@ -145,6 +145,32 @@ def make_w(w: Workload) -> torch.Tensor:
     return torch.randn(w.N, w.K, generator=g, dtype=torch.float32) * w.w_std
 
 
+def _gen_device(s: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(s)
+    return g
+
+
+def make_w_device(w: Workload, device) -> torch.Tensor:
+    """Weights drawn on the device: same seed and distribution as make_w, other values (the
+    device generator's stream).  For timing stacks whose host draw would take minutes."""
+    g = _gen_device(seed(w.config, w.layer, 1), device)
+    return torch.randn(w.N, w.K, generator=g, dtype=torch.float32, device=device) * w.w_std
+
+
+def make_x_device(w: Workload, rows: int, device, tensor_id: int = 0) -> torch.Tensor:
+    """Activations drawn on the device (normal kind, the workload's outlier channels and gain),
+    bf16 [rows, K]; tensor_id 2 gives the calibration batch."""
+    if w.x_kind != "normal":
+        raise ValueError("device draws cover the normal activation kind")
+    g = _gen_device(seed(w.config, w.layer, tensor_id), device)
+    x = torch.randn(rows, w.K, generator=g, dtype=torch.float32, device=device)
+    ch = outlier_channels(w).to(device)
+    if ch.numel():
+        x[:, ch] *= w.outlier_gain
+    return x.to(torch.bfloat16)
+
+
 def make_xcal(w: Workload) -> torch.Tensor:
     """The separate 64-token bf16 calibration batch of a workload (same distribution as x)."""
     return _draw_x(w, CALIB_TOKENS, 2).to(torch.bfloat16)
