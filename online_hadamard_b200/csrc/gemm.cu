@@ -840,8 +840,8 @@ static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch
     if (scratch && rem != 0 && KT > 1 && est_sk <= est_dp) {
         s.dp_tiles = static_cast<int>(dp);
         s.sk_units = (tiles - dp) * static_cast<int64_t>(KT);
-        s.sk_count = static_cast<int>(units);
         s.grid = units < s.sk_units ? units : s.sk_units;  // every unit gets at least one K step
+        s.sk_count = static_cast<int>(s.grid);              // the K steps go to the units launched
     } else {
         s.dp_tiles = static_cast<int>(tiles);
         s.grid = units < tiles ? units : tiles;

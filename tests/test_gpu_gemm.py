@@ -49,8 +49,8 @@ SHAPES = [
     (64, 256, 1024), (65, 130, 256), (100, 1000, 800), (128, 128, 256), (129, 300, 320),
     (256, 512, 512), (300, 520, 1056), (511, 777, 640), (1024, 2048, 2048),
     # long K, few tiles: stream-K splits every tile across many CTAs (owner + ~10-18
-    # contributors), swap-AB and 128 x 256 orientations
-    (16, 2048, 8192), (200, 1024, 8192), (70, 1100, 6144),
+    # contributors), swap-AB and CTA-pair kernels (1280 x 2048: 40 tiles on 74 pairs)
+    (16, 2048, 8192), (200, 1024, 8192), (70, 1100, 6144), (1280, 2048, 16384),
 ]
 
 
