@@ -179,6 +179,32 @@ int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * macaq_w4a4_grouped_linear -- a grouped (mixture-of-experts) W4A4 linear: E experts, each its
+ * own layer with its own per-channel scale and block-Hadamard transform folded into its weights
+ * (the method is layer-local, Abstract; the pages name MoE models among its targets), all of
+ * them computed in two launches -- a grouped transform + quantisation, then a grouped GEMM.
+ *   x         in   bf16 [T][K], the tokens grouped by expert: expert e's counts[e] rows follow
+ *                  expert e-1's (T = sum of counts)
+ *   counts    in   HOST int64 [E], tokens per expert (>= 0, zeros allowed), 1 <= E <= 128
+ *   act_mult  in   fp32 [E][K], expert e's multipliers from macaq_fold_weights; NULL: plain
+ *                  MXFP4 of x (the "pure MXFP4" baseline, no scale and no transform)
+ *   Wq, Ws    in   the experts' folded weights stacked: codes [E][N][K/2], scales the E buffers
+ *                  of macaq_scale_bytes(N, K) bytes one after another; N % 128 == 0
+ *   y         out  bf16 [T][N], row t the output of token t's expert
+ *   workspace in   at least macaq_grouped_workspace_bytes(counts, E, N, K) bytes (the activation
+ *                  codes and scales, each expert padded to whole 128-row blocks); contents on
+ *                  entry and on return unspecified; calls sharing it must be stream-ordered
+ * Experts with up to 128 tokens each run swap-AB (weights as the 128-row MMA operand); larger
+ * ones 128-token x 256-feature tiles.  y and the codes match the per-expert linear's (codes bit
+ * for bit).  Returns MACAQ_OK without launching when T == 0.
+ */
+size_t macaq_grouped_workspace_bytes(const int64_t* counts, int E, int64_t N, int64_t K);
+int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* counts, int E, int64_t K,
+                              const float* act_mult, const uint8_t* Wq, const uint8_t* Ws,
+                              int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * macaq_w4a4_linear_noalloc -- macaq_w4a4_linear for callers that cannot allocate device
  * memory.  The paper has no counterpart: it is a deployment variant of the call above.
  *

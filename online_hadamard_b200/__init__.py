@@ -24,7 +24,8 @@ from . import build as _build_mod
 __all__ = [
     "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes", "gemm_workspace_bytes",
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
-    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_linear_noalloc",
+    "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_grouped_linear",
+    "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
@@ -34,7 +35,7 @@ EXPORTED_SYMBOLS = (
     "macaq_gemm_workspace_bytes",
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
     "macaq_act_quant_plain", "macaq_mxfp4_linear", "macaq_mxfp4_gemm", "macaq_device_status",
-    "macaq_w4a4_linear_noalloc",
+    "macaq_grouped_workspace_bytes", "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc",
 )
 
 MACAQ_OK = 0
@@ -77,11 +78,14 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_mxfp4_gemm.argtypes = [p, p, i64, p, p, i64, i64, p, i32, p, sz, p]
         lib.macaq_w4a4_linear.argtypes = [p, i64, i64, p, p, p, i64, p, p, sz, p]
         lib.macaq_mxfp4_linear.argtypes = [p, i64, i64, p, p, i64, p, p, sz, p]
+        lib.macaq_grouped_workspace_bytes.argtypes = [p, i32, i64, i64]
+        lib.macaq_grouped_workspace_bytes.restype = sz
+        lib.macaq_w4a4_grouped_linear.argtypes = [p, p, i32, i64, p, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
         lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
-                     "macaq_w4a4_linear_noalloc"):
+                     "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -249,6 +253,44 @@ def macaq_mxfp4_linear(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: i
     _need(workspace, "workspace", torch.uint8)
     _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
                                              workspace.numel(), _stream(stream)), "macaq_mxfp4_linear")
+    return y
+
+
+def _counts_array(counts):
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.int64))
+    return c, ctypes.c_void_p(c.ctypes.data)
+
+
+def grouped_workspace_bytes(counts, N: int, K: int) -> int:
+    """Scratch bytes macaq_w4a4_grouped_linear needs for these per-expert token counts."""
+    c, cp = _counts_array(counts)
+    return int(load_library().macaq_grouped_workspace_bytes(cp, len(c), N, K))
+
+
+def macaq_w4a4_grouped_linear(x: torch.Tensor, counts, act_mult, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+                              y=None, workspace=None, stream=None):
+    """Grouped (mixture-of-experts) linear: x [T, K] bf16 grouped by expert, counts = tokens per
+    expert (host ints), act_mult fp32 [E, K] (None: plain MXFP4), Wq [E, N, K/2], Ws the experts'
+    scale buffers concatenated.  Returns y bf16 [T, N]."""
+    T, K = x.shape
+    c, cp = _counts_array(counts)
+    E = len(c)
+    if int(c.sum()) != T:
+        raise ValueError("counts must sum to the rows of x")
+    _need(x, "x", torch.bfloat16)
+    if act_mult is not None:
+        _need(act_mult, "act_mult", torch.float32, (E, K))
+    _need(Wq, "Wq", torch.uint8, (E, N, K // 2))
+    _need(Ws, "Ws", torch.uint8)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _need(y, "y", torch.bfloat16, (T, N))
+    need = max(grouped_workspace_bytes(c, N, K), 1)
+    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8)
+    _check(load_library().macaq_w4a4_grouped_linear(_ptr(x), cp, E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N,
+                                                    _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "macaq_w4a4_grouped_linear")
     return y
 
 

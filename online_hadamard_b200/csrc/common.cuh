@@ -36,6 +36,35 @@ inline int check_shape(int64_t rows, int64_t K) {
     return MACAQ_OK;
 }
 
+// Experts of a grouped (mixture-of-experts) linear, passed to its kernels by value.  x and y hold
+// the tokens grouped by expert; the quantised activations give every expert a segment of whole
+// 128-row blocks, so its scale atoms stay aligned; the weights are stacked [E][N][K].
+constexpr int kMaxGroups = 128;
+
+struct GroupTable {
+    int groups;
+    int rows[kMaxGroups];             // tokens of expert e
+    int x_row[kMaxGroups];            // its first row in x and y
+    int a_row[kMaxGroups + 1];        // its first row in the padded activation codes; a_row[E] = total
+    int tile_start[kMaxGroups + 1];   // its first GEMM tile; tile_start[E] = all tiles
+};
+
+struct NoGroups {};
+
+// The expert whose range [starts[e], starts[e + 1]) holds v (0 <= v < starts[E]); empty ranges
+// are skipped.
+__host__ __device__ __forceinline__ int group_of(const int* starts, int groups, int v) {
+    int lo = 0, hi = groups - 1;
+    while (lo < hi) {  // first e with starts[e + 1] > v
+        const int mid = (lo + hi) >> 1;
+        if (starts[mid + 1] > v)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    return lo;
+}
+
 inline int launch_status() {
     return cudaGetLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ECUDA;
 }

@@ -44,6 +44,8 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
                                uint8_t* Aq, uint8_t* As, cudaStream_t stream);
 int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                            cudaStream_t stream);
+int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult, uint8_t* Aq, uint8_t* As,
+                             const GroupTable& gt, cudaStream_t stream);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -88,6 +90,7 @@ struct GemmParams {
     int dp_tiles;         // tiles scheduled data-parallel (blockIdx.x + i * gridDim.x)
     int64_t sk_units;     // K steps of the remaining tiles, split evenly over the first sk_count units
     int sk_count;         // scheduling units that take part in the split (<= the units launched)
+    int64_t group_n;      // grouped linear: output features per expert (weights stacked [E][N][K])
     float* partials;      // stream-K fp32 partial accumulators, one 128 x BN slot per CTA
     uint64_t* flags;      // stream-K hand-off: one word per (partial slot, epilogue thread)
     uint64_t tag;         // this launch's value of a written flag word (unique per launch)
@@ -99,14 +102,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Store CH accumulator columns [qc, qc+CH) of P-row `prow`.
+// Store CH accumulator columns [qc, qc+CH) of P-row `prow`, in y's index space: only rows below
+// p_end and columns below q_end exist (swap-AB: P indexes y's columns and Q its rows).
 template <int CH, bool SWAP>
-__device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow, int64_t qc,
-                                            const uint32_t* r) {
-    if (prow >= prm.p_rows) return;
+__device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow, int64_t qc, const uint32_t* r,
+                                            int64_t p_end, int64_t q_end) {
+    if (prow >= p_end) return;
     if constexpr (!SWAP) {
         const int64_t base = prow * prm.ldy + qc;
-        const bool full = qc + CH <= prm.q_rows;
+        const bool full = qc + CH <= q_end;
         if (prm.y_fp32) {
             float* y = static_cast<float*>(prm.y) + base;
             if (full && (prm.ldy % 4) == 0) {
@@ -116,7 +120,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow,
             } else {
 #pragma unroll
                 for (int j = 0; j < CH; ++j)
-                    if (qc + j < prm.q_rows) y[j] = __uint_as_float(r[j]);
+                    if (qc + j < q_end) y[j] = __uint_as_float(r[j]);
             }
         } else {
             __nv_bfloat16* y = static_cast<__nv_bfloat16*>(prm.y) + base;
@@ -129,7 +133,7 @@ __device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow,
             } else {
 #pragma unroll
                 for (int j = 0; j < CH; ++j)
-                    if (qc + j < prm.q_rows) y[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                    if (qc + j < q_end) y[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
         }
     } else {
@@ -138,12 +142,12 @@ __device__ __forceinline__ void store_chunk(const GemmParams& prm, int64_t prow,
             float* y = static_cast<float*>(prm.y);
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                if (qc + j < prm.q_rows) y[(qc + j) * prm.ldy + prow] = __uint_as_float(r[j]);
+                if (qc + j < q_end) y[(qc + j) * prm.ldy + prow] = __uint_as_float(r[j]);
         } else {
             __nv_bfloat16* y = static_cast<__nv_bfloat16*>(prm.y);
 #pragma unroll
             for (int j = 0; j < CH; ++j)
-                if (qc + j < prm.q_rows) y[(qc + j) * prm.ldy + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                if (qc + j < q_end) y[(qc + j) * prm.ldy + prow] = __float2bfloat16_rn(__uint_as_float(r[j]));
         }
     }
 }
@@ -238,6 +242,7 @@ struct EpiCtx {
     int64_t prow;                 // output row (P side) of this thread
     int64_t row0;                 // first output row of this warp's 32 rows
     int64_t q0;                   // first output column (Q side) of this warp's half of the tile
+    int64_t p_end, q_end;         // exclusive limits of prow and of Q indices (see store_chunk)
     uint8_t* staging;             // this warp's 2 KB output staging buffer (TMA-store path)
 };
 
@@ -316,13 +321,59 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
         }
     }
 #pragma unroll
-    for (int c = 0; c < kHalf; c += kChunk) store_chunk<kChunk, SWAP>(prm, e.prow, e.q0 + c, v + c);
+    for (int c = 0; c < kHalf; c += kChunk) store_chunk<kChunk, SWAP>(prm, e.prow, e.q0 + c, v + c, e.p_end, e.q_end);
 }
 
-template <int BN, int STAGES, bool SWAP>
+// Where one output tile of the one-CTA kernel lives: its first P and Q operand rows (TMA
+// coordinates; the scale atoms of row r are in 128-row block r / 128), and the y coordinates of
+// its accumulator row 0 / column 0 with their exclusive limits (store_chunk's index space).
+struct TileRef {
+    int64_t p_row, q_row;
+    int64_t y_p, y_q, p_end, q_end;
+};
+
+template <int BN, bool SWAP, bool GROUPED, class GT>
+__device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& gt, int tile) {
+    TileRef t;
+    if constexpr (!GROUPED) {
+        const int pt = tile % prm.num_p_tiles, qt = tile / prm.num_p_tiles;
+        t.p_row = static_cast<int64_t>(pt) * kBM;
+        t.q_row = static_cast<int64_t>(qt) * BN;
+        t.y_p = t.p_row;
+        t.y_q = t.q_row;
+        t.p_end = prm.p_rows;
+        t.q_end = prm.q_rows;
+    } else {
+        const int e = group_of(gt.tile_start, gt.groups, tile);
+        const int local = tile - gt.tile_start[e];
+        const int64_t rows = gt.rows[e], N = prm.group_n;
+        if constexpr (!SWAP) {  // P: the expert's tokens (its padded segment), Q: its weights
+            const int ptiles = static_cast<int>((rows + kBM - 1) / kBM);
+            const int pt = local % ptiles, qt = local / ptiles;
+            t.p_row = gt.a_row[e] + static_cast<int64_t>(pt) * kBM;
+            t.q_row = e * N + static_cast<int64_t>(qt) * BN;
+            t.y_p = gt.x_row[e] + static_cast<int64_t>(pt) * kBM;  // y rows
+            t.p_end = gt.x_row[e] + rows;
+            t.y_q = static_cast<int64_t>(qt) * BN;  // y columns
+            t.q_end = N;
+        } else {  // P: the expert's weights, Q: its tokens (one tile: BN >= every expert's tokens)
+            t.p_row = e * N + static_cast<int64_t>(local) * kBM;
+            t.q_row = gt.a_row[e];
+            t.y_p = static_cast<int64_t>(local) * kBM;  // y columns
+            t.p_end = N;
+            t.y_q = gt.x_row[e];  // y rows
+            t.q_end = gt.x_row[e] + rows;
+        }
+    }
+    return t;
+}
+
+// GROUPED: a grouped (mixture-of-experts) linear; `gt` maps work tiles to experts.
+template <int BN, int STAGES, bool SWAP, bool GROUPED = false,
+          class GT = typename std::conditional<GROUPED, GroupTable, NoGroups>::type>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
-                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm) {
+                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm, const __grid_constant__ GT gt) {
     using Cfg = TileCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -369,19 +420,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             WorkIter it(prm, blockIdx.x, gridDim.x);
             Work w;
             while (!abort && it.next(prm, w)) {
-                const int pt = w.tile % prm.num_p_tiles;
-                const int qt = w.tile / prm.num_p_tiles;
-                const uint8_t* sfp = prm.sf_p + static_cast<int64_t>(pt) * (prm.kbp / 4) * 512;
+                const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, gt, w.tile);
+                const uint8_t* sfp = prm.sf_p + (t.p_row / 128) * (prm.kbp / 4) * 512;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
                     uint8_t* sb = smem + stage * Cfg::kStageBytes;
                     mbar_arrive_expect_tx(&full[stage], Cfg::kStageBytes);
-                    tma_load_2d(sb, &tmap_p, kt * kStageKBytes, pt * kBM, &full[stage]);
-                    tma_load_2d(sb + Cfg::kPBytes, &tmap_q, kt * kStageKBytes, qt * BN, &full[stage]);
+                    tma_load_2d(sb, &tmap_p, kt * kStageKBytes, static_cast<int32_t>(t.p_row), &full[stage]);
+                    tma_load_2d(sb + Cfg::kPBytes, &tmap_q, kt * kStageKBytes, static_cast<int32_t>(t.q_row),
+                                &full[stage]);
                     bulk_load(sb + Cfg::kPBytes + Cfg::kQBytes, sfp + kt * 1024, 1024, &full[stage]);
 #pragma unroll
                     for (int i = 0; i < Cfg::kQBlocks; ++i) {
-                        int qb = (qt * BN) / 128 + i;
+                        int64_t qb = t.q_row / 128 + i;
                         if (qb >= prm.q_row_blocks) qb = prm.q_row_blocks - 1;  // rows past the end: masked
                         bulk_load(sb + Cfg::kPBytes + Cfg::kQBytes + Cfg::kSFPBytes + 1024 * i,
                                   prm.sf_q + static_cast<int64_t>(qb) * (prm.kbp / 4) * 512 + kt * 1024, 1024,
@@ -464,11 +515,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         WorkIter it(prm, blockIdx.x, gridDim.x);
         Work w;
         while (!abort && it.next(prm, w)) {
-            const int pt = w.tile % prm.num_p_tiles;
-            const int qt = w.tile / prm.num_p_tiles;
+            const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, gt, w.tile);
             if (!mbar_wait(&acc_full[acc], acc_phase, &abort)) break;
             tc_fence_after();
-            const int64_t prow = static_cast<int64_t>(pt) * kBM + sub * 32 + lane;
+            const int64_t prow = t.y_p + sub * 32 + lane;
             const uint32_t tbase = tmem_base + acc * Cfg::kAccStride + half * kHalf +
                                    (static_cast<uint32_t>(sub * 32) << 16);
             uint32_t v[kHalf];
@@ -491,8 +541,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             e.slot_stride = 1;
             e.slot_off = 0;
             e.prow = prow;
-            e.row0 = static_cast<int64_t>(pt) * kBM + sub * 32;
-            e.q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
+            e.row0 = t.y_p + sub * 32;
+            e.q0 = t.y_q + half * kHalf;
+            e.p_end = t.p_end;
+            e.q_end = t.q_end;
             e.staging = staging + (warp - 2) * 2048;
             finish_item<BN, SWAP>(prm, &tmap_y, w, e, v, abort);
         }
@@ -698,6 +750,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             e.slot_off = static_cast<int>(rank);
             e.prow = row0 + lane;
             e.row0 = row0;
+            e.p_end = prm.p_rows;
+            e.q_end = prm.q_rows;
             e.q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
             e.staging = staging + (warp - 2) * 2048;
             finish_item<BN, false>(prm, &tmap_y, w, e, v, abort);
@@ -885,9 +939,27 @@ struct GemmScratch {
     size_t bytes;
 };
 
-template <int BN, int STAGES, bool SWAP>
-static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream_t stream, bool pdl) {
+// Shared-memory attributes of one kernel instantiation, set once per device.
+template <int BN, int STAGES, bool SWAP, bool GROUPED>
+static bool kernel_attributes() {
+    static int cache[64] = {0};
+    return cached_per_device(cache, [] {
+               auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP, GROUPED>;
+               const int smem = smem_bytes<BN, STAGES, SWAP>();
+               return (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
+                       cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) == cudaSuccess)
+                          ? 1
+                          : -1;
+           }) == 1;
+}
+
+// GROUPED: `groups` maps the work tiles to experts (data-parallel schedule, no scratch); the
+// operands are the padded activation codes and the stacked weights, y is [tokens][N].
+template <int BN, int STAGES, bool SWAP, bool GROUPED = false>
+static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream_t stream, bool pdl,
+                       const GroupTable* groups = nullptr, int64_t group_n = 0) {
     using Cfg = TileCfg<BN>;
+    if (GROUPED && !kernel_attributes<BN, STAGES, SWAP, GROUPED>()) return MACAQ_ECUDA;
     CUtensorMap mp, mq;
     if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, op.q_rows, op.K, BN))
         return MACAQ_ECUDA;
@@ -909,11 +981,14 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     const int ctas = grid_ctas<BN, STAGES, SWAP>();
     if (ctas < 1) return MACAQ_ECUDA;
     CUtensorMap my;
-    prm.tma_store = (!SWAP && !op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
+    prm.tma_store = (!SWAP && !GROUPED && !op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
     if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = mq;  // unused placeholder
-    const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
-    const bool scratch = ws.ptr != nullptr && ws.bytes >= streamk_bytes<BN>(ctas);
+    const int64_t tiles = GROUPED ? groups->tile_start[groups->groups]
+                                  : static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
+    if (tiles == 0) return MACAQ_OK;
+    prm.group_n = group_n;
+    const bool scratch = !GROUPED && ws.ptr != nullptr && ws.bytes >= streamk_bytes<BN>(ctas);
     const Schedule sch = plan_schedule(tiles, ctas, prm.num_k_tiles, scratch, streamk_cost_steps<BN>());
     const int64_t grid = sch.grid;
     prm.dp_tiles = sch.dp_tiles;
@@ -937,8 +1012,13 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP>, mp, mq, my, prm) != cudaSuccess)
-        return MACAQ_ECUDA;
+    if constexpr (GROUPED) {
+        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP, true>, mp, mq, my, prm, *groups) != cudaSuccess)
+            return MACAQ_ECUDA;
+    } else {
+        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP>, mp, mq, my, prm, NoGroups{}) != cudaSuccess)
+            return MACAQ_ECUDA;
+    }
     return launch_status();
 }
 
@@ -1118,6 +1198,41 @@ int run_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult, c
     return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, st, true);
 }
 
+// The group table of a grouped linear from the host token counts: tokens per expert, their rows in
+// x / y and in the padded activation codes (whole 128-row blocks per expert), and the GEMM tiles
+// per expert (swap-AB when no expert has more than 128 tokens: N / 128 weight tiles each; else
+// 128-token x 256-feature tiles).  Returns MACAQ_ESHAPE for counts out of range.
+static int build_group_table(const int64_t* counts, int E, int64_t N, GroupTable* gt, int64_t* max_rows) {
+    if (E < 1 || E > kMaxGroups) return MACAQ_ESHAPE;
+    gt->groups = E;
+    int64_t x = 0, a = 0, mx = 0;
+    for (int e = 0; e < E; ++e) {
+        if (counts[e] < 0) return MACAQ_ESHAPE;
+        gt->rows[e] = static_cast<int>(counts[e]);
+        gt->x_row[e] = static_cast<int>(x);
+        gt->a_row[e] = static_cast<int>(a);
+        x += counts[e];
+        a += (counts[e] + 127) / 128 * 128;
+        mx = counts[e] > mx ? counts[e] : mx;
+        if (a > kMaxDim) return MACAQ_ESHAPE;
+    }
+    gt->a_row[E] = static_cast<int>(a);
+    int64_t t = 0;
+    for (int e = 0; e < E; ++e) {
+        gt->tile_start[e] = static_cast<int>(t);
+        if (counts[e] > 0)
+            t += mx <= 128 ? N / 128 : (counts[e] + 127) / 128 * ((N + 255) / 256);
+    }
+    gt->tile_start[E] = static_cast<int>(t);
+    *max_rows = mx;
+    return MACAQ_OK;
+}
+
+size_t grouped_activation_bytes(int64_t padded_rows, int64_t K) {
+    return round256(static_cast<size_t>(padded_rows * (K / 2))) +
+           round256(static_cast<size_t>(scale_bytes(padded_rows, K)));
+}
+
 }  // namespace macaq
 
 using namespace macaq;
@@ -1171,4 +1286,47 @@ extern "C" int macaq_mxfp4_linear(const uint16_t* x, int64_t M, int64_t K, const
     if (workspace_bytes < macaq_linear_workspace_bytes(M, N, K)) return MACAQ_EWORKSPACE;
     return run_linear(x, M, K, nullptr, Wq, Ws, N, y, linear_workspace_layout(workspace, M, K), true,
                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t macaq_grouped_workspace_bytes(const int64_t* counts, int E, int64_t N, int64_t K) {
+    if (!counts || check_shape(1, K) || N < 128 || N % 128 != 0 || N > kMaxDim) return 0;
+    GroupTable gt;
+    int64_t mx = 0;
+    if (build_group_table(counts, E, N, &gt, &mx)) return 0;
+    return grouped_activation_bytes(gt.a_row[E], K);
+}
+
+extern "C" int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* counts, int E, int64_t K,
+                                         const float* act_mult, const uint8_t* Wq, const uint8_t* Ws, int64_t N,
+                                         uint16_t* y, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!counts || !Wq || !Ws) return MACAQ_EINVAL;
+    if (int st = check_shape(1, K)) return st;
+    if (N < 128 || N % 128 != 0 || N > kMaxDim || static_cast<int64_t>(E) * N > kMaxDim) return MACAQ_ESHAPE;
+    GroupTable gt;
+    int64_t mx = 0;
+    if (int st = build_group_table(counts, E, N, &gt, &mx)) return st;
+    if (mx == 0) return MACAQ_OK;  // no token routed to any expert
+    if (!x || !y || !workspace) return MACAQ_EINVAL;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y) || !aligned16(workspace) ||
+        (act_mult && !aligned16(act_mult)))
+        return MACAQ_EALIGN;
+    const int64_t P = gt.a_row[E];
+    if (workspace_bytes < grouped_activation_bytes(P, K)) return MACAQ_EWORKSPACE;
+    uint8_t* Aq = static_cast<uint8_t*>(workspace);
+    uint8_t* As = Aq + round256(static_cast<size_t>(P * (K / 2)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (int rc = launch_act_quant_grouped(x, K, act_mult, Aq, As, gt, st)) return rc;
+    const GemmScratch none{nullptr, 0};
+    if (mx <= 128) {  // decode-sized experts: weights on the MMA's 128-row side, tokens as N
+        return with_config(mx, [&](auto bn, auto stages, auto sw) -> int {
+            if constexpr (decltype(sw)::value) {
+                const GemmOperands op{Wq, Ws, Aq, As, E * N, P, K, y, N, 0};
+                return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, true>(op, none, st, true, &gt, N);
+            } else {
+                return MACAQ_EINVAL;  // not reached: up to 128 tokens always take a swap-AB configuration
+            }
+        });
+    }
+    const GemmOperands op{Aq, As, Wq, Ws, P, E * N, K, y, N, 0};
+    return launch_gemm<256, 4, false, true>(op, none, st, true, &gt, N);
 }

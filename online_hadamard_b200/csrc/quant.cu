@@ -217,6 +217,58 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
     }
 }
 
+// The activations of a grouped linear: thread = (group of `rpg` padded rows) x (one 32-block
+// column), as in mx_quant_kernel; each padded row belongs to one expert, whose multipliers
+// (act_mult + e K, transform mode) and source row in x it uses; padding rows past the expert's
+// tokens get zero codes and zero scales.
+template <QuantMode MODE>
+__global__ void __launch_bounds__(kQuantThreads) mx_quant_grouped_kernel(
+    const uint16_t* __restrict__ x, int64_t K, int64_t rpg, const float* __restrict__ act_mult,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const __grid_constant__ GroupTable gt) {
+    static_assert(MODE != QuantMode::kWeightFold, "activations only");
+    griddep_launch_dependents();
+    const int64_t kb_real = K / 32;
+    const int64_t kbp = padded_blocks(K);
+    const int64_t P = gt.a_row[gt.groups];
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+    const int64_t kb = item % kbp;
+    const int64_t r0 = (item / kbp) * rpg;
+    if (r0 >= P) return;
+    const int64_t r1 = r0 + rpg < P ? r0 + rpg : P;
+    const int64_t k0 = kb * 32;
+    int e = -1;
+    float2 m[16];
+    for (int64_t r = r0; r < r1; ++r) {
+        uint8_t* sc = scales + scale_offset(r, kb, kbp);
+        if (kb >= kb_real) {
+            *sc = 0;
+            continue;
+        }
+        const int er = group_of(gt.a_row, gt.groups, static_cast<int>(r));
+        const int64_t local = r - gt.a_row[er];
+        if (local >= gt.rows[er]) {  // padding row of the expert's last 128-row block
+            *reinterpret_cast<uint4*>(codes + r * (K / 2) + kb * 16) = make_uint4(0u, 0u, 0u, 0u);
+            *sc = 0;
+            continue;
+        }
+        if constexpr (MODE == QuantMode::kActTransform) {
+            if (er != e) {
+                const float4* mp = reinterpret_cast<const float4*>(act_mult + static_cast<int64_t>(er) * K + k0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 t = __ldg(mp + j);
+                    m[2 * j] = make_float2(t.x, t.y);
+                    m[2 * j + 1] = make_float2(t.z, t.w);
+                }
+            }
+        }
+        e = er;
+        RawBlock<MODE> b;
+        load_block<MODE>(x, (gt.x_row[er] + local) * K + k0, b);
+        process_block<MODE>(b, m, codes + r * (K / 2) + kb * 16, sc);
+    }
+}
+
 // Rows per thread: enough threads to fill the GPU, rows walked by each otherwise.
 static int64_t quant_rows_per_thread(int64_t R, int64_t K) {
     const int64_t cols = padded_blocks(K);
@@ -237,6 +289,20 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
     const int64_t rpg = quant_rows_per_thread(M, K);
     mx_quant_kernel<QuantMode::kActTransform><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
         x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As);
+    return launch_status();
+}
+
+int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult, uint8_t* Aq, uint8_t* As,
+                             const GroupTable& gt, cudaStream_t stream) {
+    const int64_t P = gt.a_row[gt.groups];
+    if (P == 0) return MACAQ_OK;
+    const int64_t rpg = quant_rows_per_thread(P, K);
+    if (act_mult)
+        mx_quant_grouped_kernel<QuantMode::kActTransform><<<quant_blocks(P, K, rpg), kQuantThreads, 0, stream>>>(
+            x, K, rpg, act_mult, Aq, As, gt);
+    else
+        mx_quant_grouped_kernel<QuantMode::kPlain><<<quant_blocks(P, K, rpg), kQuantThreads, 0, stream>>>(
+            x, K, rpg, nullptr, Aq, As, gt);
     return launch_status();
 }
 

@@ -97,3 +97,30 @@ def test_calibrate_scale_validation():
     assert _call("macaq_calibrate_scale", P(FAKE), 64, P(FAKE), 0, 256, P(FAKE), None) == -2
     assert _call("macaq_calibrate_scale", P(FAKE), 64, P(FAKE), 128, 200, P(FAKE), None) == -2
     assert _call("macaq_calibrate_scale", P(FAKE), 64, P(MIS), 128, 256, P(FAKE), None) == -3
+
+
+def test_grouped_linear_validation_and_sizes():
+    import numpy as np
+    P = ctypes.c_void_p
+    lib = mq.load_library()
+
+    def counts(*c):
+        a = np.array(c, dtype=np.int64)
+        return a, P(a.ctypes.data)
+
+    c, cp = counts(3, 0, 130)
+    # workspace: every expert padded to whole 128-row blocks (128 + 0 + 256 rows)
+    assert mq.grouped_workspace_bytes(c, 256, 512) == 384 * 256 + 384 * 16
+    assert mq.grouped_workspace_bytes(c, 200, 512) == 0          # N % 128 != 0
+    assert mq.grouped_workspace_bytes([-1, 4], 256, 512) == 0    # negative count
+    assert mq.grouped_workspace_bytes([1] * 129, 256, 512) == 0  # more than 128 experts
+    call = lambda cp_, E, N, x=FAKE, y=FAKE, ws=FAKE, wsb=1 << 30: lib.macaq_w4a4_grouped_linear(
+        P(x), cp_, E, 512, P(FAKE), P(FAKE), P(FAKE), N, P(y), P(ws), wsb, None)
+    assert lib.macaq_w4a4_grouped_linear(P(FAKE), None, 3, 512, P(FAKE), P(FAKE), P(FAKE), 256, P(FAKE), P(FAKE),
+                                         1 << 30, None) == -1
+    assert call(cp, 0, 256) == -2
+    assert call(cp, 3, 200) == -2
+    assert call(cp, 3, 256, x=MIS) == -3
+    assert call(cp, 3, 256, wsb=1000) == -6
+    z, zp = counts(0, 0, 0)
+    assert call(zp, 3, 256, x=0, y=0, ws=0) == 0  # no token routed: nothing to do, nothing launched
