@@ -452,6 +452,7 @@ def main():
         extra = secondary(mq, device, peaks, args)
     if not args.no_stack:
         extra["qwen3_32b_stack"] = stack_sweep(mq, device, peaks)
+        extra["qwen3_moe_grouped"] = moe_sweep(mq, device, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -553,6 +554,52 @@ def stack_sweep(mq, device, peaks, Ms=(1, 32, 512, 4096), steps=3, warmup=2):
         torch.cuda.empty_cache()
     del lin
     torch.cuda.empty_cache()
+    return res
+
+
+def moe_sweep(mq, device, peaks, token_counts=(16, 4096), steps=10, warmup=3):
+    """Grouped (mixture-of-experts) linears, Qwen3-MoE-like: 128 experts, top-8 routing, the up
+    (2048 -> 768) and down (768 -> 2048) projections; per expert its own calibrated scale and
+    folded weights.  W4A4 against plain MXFP4, graph-timed; bytes = the weights of the experts
+    that received tokens + bf16 x and y."""
+    E = wls.MOE_EXPERTS
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    res = {"experts": E, "topk": wls.MOE_TOPK}
+    for li, (name, K, N) in enumerate(wls.MOE_LINEARS):
+        Wq, Ws, am = [], [], []
+        for e in range(E):
+            wl = wls.Workload(f"moe_{name}", 6, 1, K, N, "normal", 0.01, 50.0, layer=E * li + e)
+            W = wls.make_w_device(wl, device)
+            s = mq.macaq_calibrate_scale(wls.make_x_device(wl, wls.CALIB_TOKENS, device, tensor_id=2), W)
+            q, sc, a = mq.macaq_fold_weights(W, s)
+            Wq.append(q)
+            Ws.append(sc)
+            am.append(a)
+            del W
+        Wq, Ws, am = torch.stack(Wq), torch.cat(Ws), torch.stack(am)
+        for T in token_counts:
+            counts = wls.moe_counts(T)
+            rows = sum(counts)
+            x = wls.make_x_device(wls.Workload(f"moe_{name}_x", 6, 1, K, N, "normal", 0.01, 50.0,
+                                               layer=E * li + E), rows, device)
+            y = torch.empty(rows, N, dtype=torch.bfloat16, device=device)
+            ws = torch.empty(max(mq.grouped_workspace_bytes(counts, N, K), 1), dtype=torch.uint8, device=device)
+            ms = time_loop(lambda i: mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N, y=y, workspace=ws),
+                           steps, warmup, device)
+            ms_plain = time_loop(lambda i: mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N, y=y, workspace=ws),
+                                 steps, warmup, device)
+            active = sum(1 for c in counts if c)
+            flops = 2.0 * rows * K * N
+            nbytes = active * N * K * (0.5 + 1 / 32) + 2.0 * rows * (K + N) + 4.0 * K * active
+            t_roof = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+            res[f"{name}_T{T}"] = {"routed_rows": rows, "active_experts": active, "max_rows": max(counts),
+                                    "ms": ms, "plain_mxfp4_ms": ms_plain,
+                                    "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
+                                    "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                    "linear_roofline_frac": t_roof / (ms * 1e-3)}
+            del x, y, ws
+        del Wq, Ws, am
+        torch.cuda.empty_cache()
     return res
 
 

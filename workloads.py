@@ -91,6 +91,23 @@ def stack_layer(layer: int, linear: str, M: int) -> Workload:
     raise KeyError(linear)
 
 
+# Mixture-of-experts linears (the pages name MoE models among the method's targets but give no
+# shapes): Qwen3-MoE-like experts, 128 experts of hidden 2048 / expert width 768, top-8 routing.
+MOE_EXPERTS = 128
+MOE_TOPK = 8
+MOE_LINEARS = (("up", 2048, 768), ("down", 768, 2048))
+
+
+def moe_counts(tokens: int, experts: int = MOE_EXPERTS, topk: int = MOE_TOPK, seed_: int = 6000) -> list:
+    """Tokens routed to each expert: every token picks `topk` distinct experts, with popularity
+    skewed like a learned router (Zipf-like weights 1/(rank+1) in a seeded random expert order)."""
+    g = _gen(seed_)
+    w = 1.0 / torch.arange(1, experts + 1, dtype=torch.float64)
+    w = w[torch.randperm(experts, generator=g)]
+    picks = torch.multinomial(w.expand(tokens, experts), topk, replacement=False, generator=g)
+    return torch.bincount(picks.reshape(-1), minlength=experts).tolist()
+
+
 def seed(cfg: int, layer: int, tensor_id: int) -> int:
     return 1000 * cfg + 16 * layer + tensor_id
 
