@@ -51,6 +51,13 @@ struct GroupTable {
 
 struct NoGroups {};
 
+// The grouped quantiser's threads: expert e's tokens split into runs of `rpg` rows, its runs
+// numbered from run_start[e]; run_start[E] = all runs (padding rows get no thread).
+struct RowRuns {
+    int rpg;
+    int run_start[kMaxGroups + 1];
+};
+
 // The expert whose range [starts[e], starts[e + 1]) holds v (0 <= v < starts[E]); empty ranges
 // are skipped.
 __host__ __device__ __forceinline__ int group_of(const int* starts, int groups, int v) {

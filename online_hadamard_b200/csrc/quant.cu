@@ -160,7 +160,30 @@ __device__ __forceinline__ void process_block(const RawBlock<MODE>& raw, const f
     *scale_byte = static_cast<uint8_t>(e);
 }
 
-// One thread = (group of `rpg` rows) x (one 32-block column), columns fastest; threads of
+// Quantise one 32-block column (kb) of n consecutive rows: input row in0 + i becomes output
+// row out0 + i.  Rows go two at a time, both loaded before either is used.
+template <QuantMode MODE>
+__device__ __forceinline__ void quant_rows(const void* __restrict__ in, int64_t K, int64_t in0, int64_t out0,
+                                           int64_t n, int64_t kb, int64_t kbp, const float2 (&m)[16],
+                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    const int64_t k0 = kb * 32;
+    int64_t i = 0;
+    for (; i + 1 < n; i += 2) {
+        RawBlock<MODE> b0, b1;
+        load_block<MODE>(in, (in0 + i) * K + k0, b0);
+        load_block<MODE>(in, (in0 + i + 1) * K + k0, b1);
+        const int64_t o = out0 + i;
+        process_block<MODE>(b0, m, codes + o * (K / 2) + kb * 16, scales + scale_offset(o, kb, kbp));
+        process_block<MODE>(b1, m, codes + (o + 1) * (K / 2) + kb * 16, scales + scale_offset(o + 1, kb, kbp));
+    }
+    if (i < n) {
+        RawBlock<MODE> b0;
+        load_block<MODE>(in, (in0 + i) * K + k0, b0);
+        process_block<MODE>(b0, m, codes + (out0 + i) * (K / 2) + kb * 16, scales + scale_offset(out0 + i, kb, kbp));
+    }
+}
+
+// One thread = (run of `rpg` rows) x (one 32-block column), columns fastest; threads of
 // padded block columns (kb >= K/32) write the zero scale bytes of their rows.
 template <QuantMode MODE>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
@@ -174,9 +197,9 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
     const int64_t kb = item % kbp;
     const int64_t r0 = (item / kbp) * rpg;
     if (r0 >= R) return;
-    const int64_t r1 = r0 + rpg < R ? r0 + rpg : R;
+    const int64_t n = r0 + rpg < R ? rpg : R - r0;
     if (kb >= kb_real) {
-        for (int64_t r = r0; r < r1; ++r) scales[scale_offset(r, kb, kbp)] = 0;
+        for (int64_t r = r0; r < r0 + n; ++r) scales[scale_offset(r, kb, kbp)] = 0;
         return;
     }
     const int64_t k0 = kb * 32;
@@ -202,77 +225,53 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(
             }
         }
     }
-    int64_t r = r0;
-    for (; r + 1 < r1; r += 2) {
-        RawBlock<MODE> b0, b1;
-        load_block<MODE>(in, r * K + k0, b0);
-        load_block<MODE>(in, (r + 1) * K + k0, b1);
-        process_block<MODE>(b0, m, codes + r * (K / 2) + kb * 16, scales + scale_offset(r, kb, kbp));
-        process_block<MODE>(b1, m, codes + (r + 1) * (K / 2) + kb * 16, scales + scale_offset(r + 1, kb, kbp));
-    }
-    if (r < r1) {
-        RawBlock<MODE> b0;
-        load_block<MODE>(in, r * K + k0, b0);
-        process_block<MODE>(b0, m, codes + r * (K / 2) + kb * 16, scales + scale_offset(r, kb, kbp));
-    }
+    quant_rows<MODE>(in, K, r0, r0, n, kb, kbp, m, codes, scales);
 }
 
-// The activations of a grouped linear: thread = (group of `rpg` padded rows) x (one 32-block
-// column), as in mx_quant_kernel; each padded row belongs to one expert, whose multipliers
-// (act_mult + e K, transform mode) and source row in x it uses; padding rows past the expert's
-// tokens get zero codes and zero scales.
+// The activations of a grouped linear: thread = (run of `rpg` tokens of one expert) x (one
+// 32-block column).  Expert e's token t (row x_row[e] + t of x) becomes row a_row[e] + t of the
+// padded codes, quantised with the expert's own multipliers (act_mult + e K, transform mode).
+// The padding rows up to the next 128-row boundary are left as they are: they reach only rows
+// of the GEMM's output tile that are never stored.
 template <QuantMode MODE>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_grouped_kernel(
-    const uint16_t* __restrict__ x, int64_t K, int64_t rpg, const float* __restrict__ act_mult,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const __grid_constant__ GroupTable gt) {
+    const uint16_t* __restrict__ x, int64_t K, const float* __restrict__ act_mult, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, const __grid_constant__ GroupTable gt, const __grid_constant__ RowRuns rr) {
     static_assert(MODE != QuantMode::kWeightFold, "activations only");
     griddep_launch_dependents();
-    const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
-    const int64_t P = gt.a_row[gt.groups];
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
     const int64_t kb = item % kbp;
-    const int64_t r0 = (item / kbp) * rpg;
-    if (r0 >= P) return;
-    const int64_t r1 = r0 + rpg < P ? r0 + rpg : P;
-    const int64_t k0 = kb * 32;
-    int e = -1;
-    float2 m[16];
-    for (int64_t r = r0; r < r1; ++r) {
-        uint8_t* sc = scales + scale_offset(r, kb, kbp);
-        if (kb >= kb_real) {
-            *sc = 0;
-            continue;
-        }
-        const int er = group_of(gt.a_row, gt.groups, static_cast<int>(r));
-        const int64_t local = r - gt.a_row[er];
-        if (local >= gt.rows[er]) {  // padding row of the expert's last 128-row block
-            *reinterpret_cast<uint4*>(codes + r * (K / 2) + kb * 16) = make_uint4(0u, 0u, 0u, 0u);
-            *sc = 0;
-            continue;
-        }
-        if constexpr (MODE == QuantMode::kActTransform) {
-            if (er != e) {
-                const float4* mp = reinterpret_cast<const float4*>(act_mult + static_cast<int64_t>(er) * K + k0);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 t = __ldg(mp + j);
-                    m[2 * j] = make_float2(t.x, t.y);
-                    m[2 * j + 1] = make_float2(t.z, t.w);
-                }
-            }
-        }
-        e = er;
-        RawBlock<MODE> b;
-        load_block<MODE>(x, (gt.x_row[er] + local) * K + k0, b);
-        process_block<MODE>(b, m, codes + r * (K / 2) + kb * 16, sc);
+    const int run = static_cast<int>(item / kbp);
+    if (run >= rr.run_start[gt.groups]) return;
+    const int e = group_of(rr.run_start, gt.groups, run);
+    const int64_t t0 = static_cast<int64_t>(run - rr.run_start[e]) * rr.rpg;
+    const int64_t n = t0 + rr.rpg < gt.rows[e] ? rr.rpg : gt.rows[e] - t0;
+    const int64_t out0 = gt.a_row[e] + t0;
+    if (kb >= K / 32) {
+        for (int64_t r = out0; r < out0 + n; ++r) scales[scale_offset(r, kb, kbp)] = 0;
+        return;
     }
+    float2 m[16];
+    if constexpr (MODE == QuantMode::kActTransform) {
+        const float4* mp = reinterpret_cast<const float4*>(act_mult + static_cast<int64_t>(e) * K + kb * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 t = __ldg(mp + j);
+            m[2 * j] = make_float2(t.x, t.y);
+            m[2 * j + 1] = make_float2(t.z, t.w);
+        }
+    }
+    quant_rows<MODE>(x, K, gt.x_row[e] + t0, out0, n, kb, kbp, m, codes, scales);
 }
 
 // Rows per thread: enough threads to fill the GPU, rows walked by each otherwise.
+// The threads one wave of the transform kernel holds: 4 CTAs of 128 per SM (128 registers).
+static int64_t quant_thread_target() { return static_cast<int64_t>(sm_count()) * 16 * 32; }
+
 static int64_t quant_rows_per_thread(int64_t R, int64_t K) {
     const int64_t cols = padded_blocks(K);
-    const int64_t target = static_cast<int64_t>(sm_count()) * 16 * 32;
+    const int64_t target = quant_thread_target();
     int64_t rpg = (R * cols + target - 1) / target;
     if (rpg < 1) rpg = 1;
     return rpg;
@@ -294,15 +293,39 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
 
 int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult, uint8_t* Aq, uint8_t* As,
                              const GroupTable& gt, cudaStream_t stream) {
-    const int64_t P = gt.a_row[gt.groups];
-    if (P == 0) return MACAQ_OK;
-    const int64_t rpg = quant_rows_per_thread(P, K);
+    int64_t tokens = 0;
+    for (int e = 0; e < gt.groups; ++e) tokens += gt.rows[e];
+    if (tokens == 0) return MACAQ_OK;
+    // The shortest runs that keep the grid within one resident wave: a second wave would share
+    // the SMs with the GEMM's CTAs, which the programmatic launch makes resident as soon as
+    // first-wave CTAs leave.  The run count falls as runs lengthen, and runs as long as the
+    // largest expert give each expert one run, the fewest possible.
+    const int64_t kbp = padded_blocks(K);
+    int max_rows = 0;
+    for (int e = 0; e < gt.groups; ++e) max_rows = gt.rows[e] > max_rows ? gt.rows[e] : max_rows;
+    auto runs = [&](int rpg) {
+        int64_t n = 0;
+        for (int e = 0; e < gt.groups; ++e) n += (gt.rows[e] + rpg - 1) / rpg;
+        return n;
+    };
+    int lo = static_cast<int>(quant_rows_per_thread(tokens, K)), hi = max_rows;
+    if (lo > hi) lo = hi;
+    while (lo < hi) {  // first rpg in [lo, hi] whose grid fits; hi if none does
+        const int mid = lo + (hi - lo) / 2;
+        if (kbp * runs(mid) <= quant_thread_target()) hi = mid;
+        else lo = mid + 1;
+    }
+    RowRuns rr;
+    rr.rpg = lo;
+    rr.run_start[0] = 0;
+    for (int e = 0; e < gt.groups; ++e) rr.run_start[e + 1] = rr.run_start[e] + (gt.rows[e] + lo - 1) / lo;
+    const int64_t items = kbp * rr.run_start[gt.groups];
+    const unsigned blocks = static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
     if (act_mult)
-        mx_quant_grouped_kernel<QuantMode::kActTransform><<<quant_blocks(P, K, rpg), kQuantThreads, 0, stream>>>(
-            x, K, rpg, act_mult, Aq, As, gt);
+        mx_quant_grouped_kernel<QuantMode::kActTransform><<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq,
+                                                                                               As, gt, rr);
     else
-        mx_quant_grouped_kernel<QuantMode::kPlain><<<quant_blocks(P, K, rpg), kQuantThreads, 0, stream>>>(
-            x, K, rpg, nullptr, Aq, As, gt);
+        mx_quant_grouped_kernel<QuantMode::kPlain><<<blocks, kQuantThreads, 0, stream>>>(x, K, nullptr, Aq, As, gt, rr);
     return launch_status();
 }
 

@@ -1,8 +1,10 @@
 """GPU parity of the grouped (mixture-of-experts) W4A4 linear.  Each expert is its own linear
 layer ("MACaQ", Abstract: layer-local), so the reference is the per-expert path: the codes the
-grouped quantiser writes equal the per-expert quantiser's bit for bit (padding rows zero), and y
-matches the oracle's fp64 contraction of those codes with each expert's folded weights within
-the GEMM tolerance, for the transformed and the plain (NULL multiplier) activations."""
+grouped quantiser writes equal the per-expert quantiser's bit for bit, and y matches the
+oracle's fp64 contraction of those codes with each expert's folded weights within the GEMM
+tolerance, for the transformed and the plain (NULL multiplier) activations.  The padding rows of
+each expert's 128-row segment are never written: the workspace starts as 0xFF (NaN scale bytes,
+-6 codes), so a padding row that reached a stored output would show as a NaN in y."""
 import numpy as np
 import pytest
 import torch
@@ -54,10 +56,11 @@ def test_grouped_matches_per_expert(mq, name, counts, N, K, plain):
     Wq, Ws, am = _experts(mq, E, N, K, seed=E * 31 + N + K)
     g = torch.Generator().manual_seed(T + K)
     x = (torch.randn(T, K, generator=g) * 2).to(torch.bfloat16).cuda()
-    ws = torch.full((mq.grouped_workspace_bytes(counts, N, K),), 0x5A, dtype=torch.uint8, device="cuda")
+    ws = torch.full((mq.grouped_workspace_bytes(counts, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
     y = mq.macaq_w4a4_grouped_linear(x, counts, None if plain else am, Wq, Ws, N, workspace=ws)
     torch.cuda.synchronize()
     assert mq.macaq_device_status() == 0
+    assert bool(torch.isfinite(y.float()).all())
     sb = mq.scale_bytes(N, K)
     P = sum((c + 127) // 128 * 128 for c in counts)
     Aq_all = ws[:P * K // 2].view(P, K // 2)
@@ -73,8 +76,6 @@ def test_grouped_matches_per_expert(mq, name, counts, N, K, plain):
             assert torch.equal(Aq_all[a_row:a_row + c], Aq)  # codes bit for bit
             Asr = layout.tiled_to_rowmajor(gu.to_np(As), c, K)
             assert np.array_equal(As_rows[a_row:a_row + c], Asr)
-            pad = (c + 127) // 128 * 128
-            assert torch.count_nonzero(Aq_all[a_row + c:a_row + pad]).item() == 0  # padding rows
             ref = oracle.mx_gemm(gu.to_np(Aq), Asr, gu.to_np(Wq[e]),
                                  layout.tiled_to_rowmajor(gu.to_np(Ws[e * sb:(e + 1) * sb]), N, K))
             err = gu.rel_fro(gu.to_np(y[x_row:x_row + c].float()), gu.bf16_round(ref))
