@@ -297,8 +297,12 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
     if constexpr (!SWAP && kHalf % 32 == 0) {
         if (prm.tma_store) {
             // bf16 tile through this warp's 2 KB staging buffer (32 rows x 64 B, 64-byte
-            // swizzle: conflict-free 16-byte writes) and a TMA store per 32 columns; the
-            // store clips rows and columns past the matrix edge.
+            // swizzle: conflict-free 16-byte writes), then per 32 columns either a TMA store
+            // (which clips at the matrix edge) when all 32 rows are below p_end, or -- where
+            // the rows past p_end belong to someone else (the next expert of a grouped linear)
+            // -- 16-byte stores of whole 64-byte row pieces, 8 rows per warp instruction,
+            // each row checked against p_end.
+            const bool whole = e.row0 + 32 <= e.p_end;
 #pragma unroll
             for (int c = 0; c < kHalf; c += 32) {
                 if (e.lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
@@ -310,11 +314,30 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
                         make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
                                    pack_bf16x2(r[6], r[7]));
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (e.lane == 0) {
-                    tma_store_2d(tmap_y, e.staging, static_cast<int32_t>(e.q0 + c), static_cast<int32_t>(e.row0));
-                    bulk_commit_group();
+                if (whole) {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (e.lane == 0) {
+                        tma_store_2d(tmap_y, e.staging, static_cast<int32_t>(e.q0 + c), static_cast<int32_t>(e.row0));
+                        bulk_commit_group();
+                    }
+                } else {
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = i * 8 + (e.lane >> 2), q4 = e.lane & 3;
+                        const int64_t row = e.row0 + rr, col = e.q0 + c + 8 * q4;
+                        if (row >= e.p_end) continue;
+                        const uint4 val = *reinterpret_cast<const uint4*>(e.staging + rr * 64 + 16 * (q4 ^ ((rr >> 1) & 3)));
+                        uint16_t* dst = static_cast<uint16_t*>(prm.y) + row * prm.ldy + col;
+                        if (col + 8 <= e.q_end) {
+                            *reinterpret_cast<uint4*>(dst) = val;
+                        } else {
+                            const uint16_t* h = reinterpret_cast<const uint16_t*>(&val);
+                            for (int j = 0; j < 8; ++j)
+                                if (col + j < e.q_end) dst[j] = h[j];
+                        }
+                    }
                 }
             }
             return;
@@ -819,11 +842,11 @@ static int smem_bytes() {
 }
 
 // Tensor map of the bf16 output [rows][cols]: 32 x 32 boxes, 64-byte swizzle.
-static bool make_out_map(CUtensorMap* map, void* y, int64_t rows, int64_t cols) {
+static bool make_out_map(CUtensorMap* map, void* y, int64_t rows, int64_t cols, int64_t ldy) {
     auto encode = tensor_map_encoder();
     if (!encode) return false;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldy * 2)};
     cuuint32_t box[2] = {32, 32};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
@@ -981,8 +1004,11 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     const int ctas = grid_ctas<BN, STAGES, SWAP>();
     if (ctas < 1) return MACAQ_ECUDA;
     CUtensorMap my;
-    prm.tma_store = (!SWAP && !GROUPED && !op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
-    if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows)) return MACAQ_ECUDA;
+    // y is [p_rows][q_rows], or for a grouped linear [tokens][group_n]
+    const int64_t y_rows = GROUPED ? groups->x_row[groups->groups - 1] + groups->rows[groups->groups - 1] : op.p_rows;
+    const int64_t y_cols = GROUPED ? group_n : op.q_rows;
+    prm.tma_store = (!SWAP && !op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
+    if (prm.tma_store && !make_out_map(&my, op.y, y_rows, y_cols, op.ldy)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = mq;  // unused placeholder
     const int64_t tiles = GROUPED ? groups->tile_start[groups->groups]
                                   : static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
@@ -1080,7 +1106,7 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     prm.num_k_tiles = static_cast<int>((op.K + kStageK - 1) / kStageK);
     prm.q_row_blocks = static_cast<int>((op.q_rows + 127) / 128);
     prm.tma_store = (!op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
-    if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows)) return MACAQ_ECUDA;
+    if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows, op.ldy)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = ma;  // unused placeholder
 
     const int64_t tiles = static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
