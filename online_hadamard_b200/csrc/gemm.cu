@@ -586,31 +586,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64):
 //   - each CTA TMA-loads its own 128 rows of the activation tile and its own 128 rows of the
 //     weight tile per K step, so a weight panel crosses L2 -> SM once per pair instead of once
-//     per CTA (35 KB per CTA per K step instead of 51 KB);
-//   - each CTA loads the scales of its 128 activation rows and of all 256 weight rows;
-//     tcgen05.cp.cta_group::2 moves them into the same TMEM columns of both CTAs;
-//   - all loads of both CTAs complete on the even CTA's "full" barrier; its single MMA thread
-//     issues the pair MMAs and multicasts each stage's release to both CTAs' "empty" barriers
-//     and each tile's completion to both "acc_full" barriers;
+//     per CTA (32 KB of codes per CTA per K step instead of 48 KB), completing on the even
+//     CTA's "full" barrier;
+//   - each CTA also loads the K step's scale atoms (its 128 activation rows, all 256 weight
+//     rows: 3 KB) into the same stage, completing on its own "sf_smem" barrier.  Four "scale
+//     warps" per CTA, one per TMEM sub-partition, move them from shared memory into that
+//     stage's TMEM scale buffer with tcgen05.st, in the layout a 32x128b.warpx4 copy gives
+//     (each lane's four columns hold 16 bytes of an atom, repeated in every sub-partition),
+//     and arrive on the even CTA's "sf_full" barrier.  Issuing the copies as tcgen05.cp from
+//     the MMA thread instead puts six copies per K step into the MMA issue stream, about a
+//     third of the mainloop on these shapes;
+//   - the even CTA's single MMA thread waits for both barriers, issues the pair MMAs and
+//     multicasts each stage's release to both CTAs' "empty" barriers (which also free the
+//     stage's TMEM scale buffer) and each tile's completion to both "acc_full" barriers;
 //   - each CTA's eight epilogue warps drain its 128 accumulator rows and release them on the
 //     even CTA's "acc_empty" barrier (512 arrivals: both CTAs).
+// 512 threads: warp 0 producer, warp 1 TMEM allocation and MMA issue, warps 2-3 idle, warps
+// 4-7 scale warps, warps 8-15 epilogue.  The first two warpgroups give registers to the
+// epilogue's (setmaxnreg), which holds 128 accumulator columns per thread.
 // Scheduling (data-parallel waves then stream-K) works on pairs; partial-sum slots stay per CTA.
 constexpr int kPairStages = 5;
+constexpr int kPairThreads = 512;
+constexpr int kPairLaunchRegs = 65536 / kPairThreads;  // registers per thread at launch
+constexpr int kPairLowRegs = 80;                        // producer, MMA and scale warpgroups
+constexpr int kPairEpiRegs = 176;                       // epilogue warpgroups
+static_assert(2 * 128 * kPairLowRegs + 2 * 128 * kPairEpiRegs <= kPairThreads * kPairLaunchRegs,
+              "the register split must fit in the registers the block is launched with");
 struct PairCfg {
     static constexpr int kABytes = 128 * kStageKBytes;     // this CTA's 128 activation rows
     static constexpr int kBBytes = 128 * kStageKBytes;     // this CTA's 128 weight rows
     static constexpr int kSFABytes = 1024;                 // 128 rows x 8 blocks
     static constexpr int kSFBBytes = 2048;                 // all 256 weight rows x 8 blocks
-    static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+    static constexpr int kCodeBytes = kABytes + kBBytes;
+    static constexpr int kStageBytes = kCodeBytes + kSFABytes + kSFBBytes;
     static constexpr int kSFBufCols = 8 + 16;              // SFA 2 groups x 4, SFB 2 groups x 8
     static constexpr int kSFBase = 256;                    // after the 256-column accumulator
     static constexpr int kTmemCols = 512;
     static_assert(kStageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
-    static_assert(kSFBase + 2 * kSFBufCols <= kTmemCols, "tensor memory budget");
+    static_assert(kSFBase + kPairStages * kSFBufCols <= kTmemCols, "tensor memory budget");
 };
 
 template <int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                           const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm) {
@@ -621,7 +638,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* staging = smem + STAGES * Cfg::kStageBytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
     uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
+    uint64_t* sf_smem = empty + STAGES;
+    uint64_t* sf_full = sf_smem + STAGES;
+    uint64_t* acc_full = sf_full + STAGES;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
@@ -636,6 +655,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_smem[s], 1);
+            mbar_init(&sf_full[s], 8);  // four scale warps in each CTA
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * kEpiThreads);
@@ -656,6 +677,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     int abort = 0;
 
+    if (warp < 8) setmaxnreg_dec<kPairLowRegs>();
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------- producer (both CTAs)
@@ -672,14 +694,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kt = w.k0; kt < w.k1; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
                     uint8_t* sb = smem + stage * Cfg::kStageBytes;
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kStageBytes);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * Cfg::kCodeBytes);
                     tma_load_2d_pair(sb, &tmap_a, kt * kStageKBytes, a_row, &full[stage]);
                     tma_load_2d_pair(sb + Cfg::kABytes, &tmap_b, kt * kStageKBytes, b_row, &full[stage]);
-                    uint8_t* sf = sb + Cfg::kABytes + Cfg::kBBytes;
                     // scale atoms: 1 KB (two 512-byte atoms) per 128 rows per K step, as uint32 boxes
-                    tma_load_2d_pair(sf, &tmap_sfa, kt * 256, 2 * pt + static_cast<int>(rank), &full[stage]);
-                    tma_load_2d_pair(sf + 1024, &tmap_sfb, kt * 256, 2 * qt, &full[stage]);
-                    tma_load_2d_pair(sf + 2048, &tmap_sfb, kt * 256, 2 * qt + 1, &full[stage]);
+                    uint8_t* sf = sb + Cfg::kCodeBytes;
+                    mbar_arrive_expect_tx(&sf_smem[stage], Cfg::kSFABytes + Cfg::kSFBBytes);
+                    tma_load_2d(sf, &tmap_sfa, kt * 256, 2 * pt + static_cast<int>(rank), &sf_smem[stage]);
+                    tma_load_2d(sf + 1024, &tmap_sfb, kt * 256, 2 * qt, &sf_smem[stage]);
+                    tma_load_2d(sf + 2048, &tmap_sfb, kt * 256, 2 * qt + 1, &sf_smem[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -695,7 +718,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t acc_phase = 0;
-            uint32_t sfbuf = 0;
             WorkIter it(prm, pair, pairs);
             Work w;
             while (!abort && it.next(prm, w)) {
@@ -703,20 +725,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 acc_phase ^= 1u;
                 tc_fence_after();
                 for (int kt = w.k0; kt < w.k1; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, &abort)) break;  // no tcgen05 fence: see above
+                    if (!mbar_wait(&full[stage], phase, &abort)) break;
+                    if (!mbar_wait(&sf_full[stage], phase, &abort)) break;
+                    tc_fence_after();  // the scale warps' tcgen05.st precede these MMAs
                     const uint32_t sp = smem_u32(smem + stage * Cfg::kStageBytes);
                     const uint32_t sq = sp + Cfg::kABytes;
-                    const uint32_t ssfa = sq + Cfg::kBBytes;
-                    const uint32_t ssfb = ssfa + Cfg::kSFABytes;
-                    const uint32_t tsfa = tmem_base + Cfg::kSFBase + sfbuf * Cfg::kSFBufCols;
+                    const uint32_t tsfa = tmem_base + Cfg::kSFBase + stage * Cfg::kSFBufCols;
                     const uint32_t tsfb = tsfa + 8;
-                    sfbuf ^= 1u;
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        tc_cp_sf_pair(tsfa + 4 * g, desc_sf(ssfa + 512 * g));
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) tc_cp_sf_pair(tsfb + 8 * g + 4 * i, desc_sf(ssfb + 1024 * i + 512 * g));
-                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t g = j >> 1;
@@ -726,7 +741,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tc_mma_mxf4_pair(tmem_base, desc_sw128(sp + 32 * j), desc_sw128(sq + 32 * j),
                                          idesc | (id << 29) | (id << 4), sfa, sfb, (kt != w.k0 || j != 0) ? 1u : 0u);
                     }
-                    tc_commit_pair(&empty[stage]);  // frees the stage in both CTAs
+                    tc_commit_pair(&empty[stage]);  // frees the stage and its scale buffer in both CTAs
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -736,12 +751,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 4 && warp < 8) {
+        // -------------------------------------------------------- scale warps (both CTAs)
+        // Warp (4 + sub) writes TMEM lanes 32 sub .. 32 sub + 31 of each stage's scale buffer:
+        // columns 0-7 the activation atoms (rows of this CTA), 8-23 the weight atoms (all 256
+        // rows of the tile), ordered as the MMA's scale addresses expect.  The stage's smem
+        // was refilled only after its previous MMAs completed, so its TMEM buffer is free too.
+        const int sub = warp & 3;
+        int stage = 0;
+        uint32_t phase = 0;
+        WorkIter it(prm, pair, pairs);
+        Work w;
+        while (!abort && it.next(prm, w)) {
+            for (int kt = w.k0; kt < w.k1; ++kt) {
+                if (!mbar_wait(&sf_smem[stage], phase, &abort)) break;
+                const uint8_t* sf = smem + stage * Cfg::kStageBytes + Cfg::kCodeBytes + lane * 16;
+                uint4 v[6];
+                v[0] = *reinterpret_cast<const uint4*>(sf);          // SFA atom 0
+                v[1] = *reinterpret_cast<const uint4*>(sf + 512);    // SFA atom 1
+                v[2] = *reinterpret_cast<const uint4*>(sf + 1024);   // SFB rows 0-127, atom 0
+                v[3] = *reinterpret_cast<const uint4*>(sf + 2048);   // SFB rows 128-255, atom 0
+                v[4] = *reinterpret_cast<const uint4*>(sf + 1536);   // SFB rows 0-127, atom 1
+                v[5] = *reinterpret_cast<const uint4*>(sf + 2560);   // SFB rows 128-255, atom 1
+                const uint32_t taddr =
+                    tmem_base + Cfg::kSFBase + stage * Cfg::kSFBufCols + (static_cast<uint32_t>(sub * 32) << 16);
+                tmem_st16(taddr, reinterpret_cast<const uint32_t*>(&v[0]));
+                tmem_st8(taddr + 16, reinterpret_cast<const uint32_t*>(&v[4]));
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(&sf_full[stage]);
+                    else
+                        mbar_arrive_cluster(&sf_full[stage], 0);
+                }
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp >= 8) {
         // ----------------------------------------------------------- epilogue (both CTAs)
+        setmaxnreg_inc<kPairEpiRegs>();
         constexpr int kHalf = BN / 2;
         const int sub = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const int etid = threadIdx.x - 64;
+        const int half = (warp - 8) >> 2;
+        const int etid = threadIdx.x - 256;
         uint32_t acc_phase = 0;
         WorkIter it(prm, pair, pairs);
         Work w;
@@ -776,7 +833,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             e.p_end = prm.p_rows;
             e.q_end = prm.q_rows;
             e.q0 = static_cast<int64_t>(qt) * BN + half * kHalf;
-            e.staging = staging + (warp - 2) * 2048;
+            e.staging = staging + (warp - 8) * 2048;
             finish_item<BN, false>(prm, &tmap_y, w, e, v, abort);
         }
         if (lane == 0) bulk_wait_group<0>();
@@ -1051,7 +1108,7 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
 // Kernel configuration for M rows of activations: swap-AB with the narrowest N that holds
 // the tokens for M <= 128, 128 x 256 tiles above.  `f` is called with the configuration.
 static int pair_smem_bytes() {
-    return kPairStages * PairCfg::kStageBytes + kStagingBytes + (2 * kPairStages + 2) * 8 + 16 + 1024;
+    return kPairStages * PairCfg::kStageBytes + kStagingBytes + (4 * kPairStages + 2) * 8 + 16 + 1024;
 }
 
 static int gemm_pairs_query();
@@ -1065,11 +1122,19 @@ static int gemm_pairs() {
 static int gemm_pairs_query() {
     auto kernel = mxf4_gemm_pair_kernel<kPairStages>;
     const int smem = pair_smem_bytes();
+    // setmaxnreg.inc takes registers from those the block was launched with: a kernel built
+    // with fewer than the split assumes would wait forever there, so it is never launched.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    if (fa.numRegs * kPairThreads < 2 * 128 * kPairLowRegs + 2 * 128 * kPairEpiRegs) return 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sm_count() & ~1));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1127,7 +1192,7 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * grid_pairs));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = pair_smem_bytes();
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
