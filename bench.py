@@ -465,7 +465,7 @@ def main():
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4 (e2m1 x e2m1, ue8m0 scales, fp32 accumulate, bf16 out)", "data": "synthetic",
             "config": headline_config(wl, world, f"inputs rotated over {layer.copies} copies (> 3x L2)"),
-            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<6> (2-CTA 256x256 tiles)", "achieved": gemm_tflops,
+            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<5> (2-CTA 256x256 tiles, scale warps)", "achieved": gemm_tflops,
                          "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
                          "ms_per_launch": ms_gemm},

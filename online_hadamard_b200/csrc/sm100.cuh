@@ -272,15 +272,6 @@ __device__ __forceinline__ void setmaxnreg_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// 16-byte read-only load through the non-coherent path (data written by earlier grids only).
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 // ------------------------------------------------------------- CTA pairs (cta_group::2)
 //
 // Two CTAs of a cluster on the two SMs of a TPC share one MMA: the even CTA (rank 0) issues
