@@ -15,16 +15,21 @@
 //              weight rows fill the 128-row MMA and a few tokens form a narrow N.
 //   warp 0     producer: TMA (128-byte swizzle) loads of both code tiles and linear bulk
 //              copies of the matching 512-byte scale atoms into a STAGES-deep ring.
-//   warp 1     allocates tensor memory; one lane issues, per stage, tcgen05.cp of the
-//              scale atoms into TMEM and four tcgen05.mma (K = 64 each), then commits the
-//              stage back to the producer and, per tile, the accumulator to the epilogue.
-//   warps 2-9  epilogue: two warps per TMEM sub-partition (warp w reads lanes of
+//   warp 1     allocates tensor memory; one lane issues, per stage, four tcgen05.mma
+//              (K = 64 each), then commits the stage back to the producer and, per tile,
+//              the accumulator to the epilogue.
+//   warps 2-3  idle.
+//   warps 4-7  scale warps, one per TMEM sub-partition: per stage they move the scale atoms
+//              from shared memory into the stage's own TMEM scale buffer with tcgen05.st (the
+//              MMA thread issues no tcgen05.cp) and signal the MMA thread.
+//   warps 8-15 epilogue: two warps per TMEM sub-partition (warp w reads lanes of
 //              sub-partition w % 4, one half of the tile's columns each) copy the fp32
 //              accumulator into registers, hand the TMEM back to the MMA warp at once, then
 //              convert and store y, so the next tile's mainloop overlaps the stores.
-//   Scale factors are double-buffered in TMEM (alternating per k-tile), so the copy for
-//   k-tile t+1 never writes columns the MMAs of k-tile t still read.  Accumulators are
-//   double-buffered too when BN <= 128.  All waits are bounded (see sm100.cuh).
+//   Each pipeline stage has its own TMEM scale buffer, free again once the stage's MMAs
+//   have completed.  Accumulators are double-buffered when BN <= 128.  The first two
+//   warpgroups hand registers to the epilogue's (setmaxnreg).  All waits are bounded (see
+//   sm100.cuh).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -50,8 +55,13 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
 constexpr int kStageKBytes = 128;  // code bytes per row per stage
-constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kGemmThreads = 512;  // producer, MMA, 2 idle, 4 scale and 8 epilogue warps
 constexpr int kEpiThreads = 256;
+constexpr int kLaunchRegs = 65536 / kGemmThreads;  // registers per thread at launch
+constexpr int kLowRegs = 80;                        // producer, MMA and scale warpgroups
+constexpr int kEpiRegs = 176;                       // epilogue warpgroups
+static_assert(2 * 128 * kLowRegs + 2 * 128 * kEpiRegs <= kGemmThreads * kLaunchRegs,
+              "the register split must fit in the registers the block is launched with");
 constexpr int kStagingBytes = 8 * 2048;  // output staging of the TMA-store epilogue
 // Critical-path cost of a stream-K fix-up, in K steps of the tile: a 128 x 256 fp32 partial
 // round trip through L2 (measured ~24 steps of a 128 x 256 tile) or a narrow swap-AB one.
@@ -70,13 +80,18 @@ struct TileCfg {
     static constexpr int kAccStride = ((BN + 31) / 32) * 32;
     static constexpr int kSFQColsPerGroup = 4 * kQBlocks;
     static constexpr int kSFBufCols = 8 + 2 * kSFQColsPerGroup;    // P: 2 groups x 4, then Q
-    static constexpr int kSFBase = kNumAcc * kAccStride;           // two scale buffers follow
-    static constexpr int kColsUsed = kSFBase + 2 * kSFBufCols;
-    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
-                                   : kColsUsed <= 256 ? 256 : 512;
-    static_assert(kColsUsed <= 512, "tensor memory budget");
+    static constexpr int kSFBase = kNumAcc * kAccStride;           // one scale buffer per stage follows
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
     static_assert(kStageBytes % 1024 == 0, "stage alignment for the 128-byte swizzle");
+};
+
+// Tensor memory of a configuration: accumulators, then one scale buffer per stage.
+template <int BN, int STAGES>
+struct TileTmem {
+    static constexpr int kColsUsed = TileCfg<BN>::kSFBase + STAGES * TileCfg<BN>::kSFBufCols;
+    static constexpr int kCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                               : kColsUsed <= 256 ? 256 : 512;
+    static_assert(kColsUsed <= 512, "tensor memory budget");
 };
 
 struct GemmParams {
@@ -398,12 +413,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mxf4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm, const __grid_constant__ GT gt) {
     using Cfg = TileCfg<BN>;
+    constexpr int kTmemCols = TileTmem<BN, STAGES>::kCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* staging = smem + STAGES * Cfg::kStageBytes;  // per epilogue warp: 32 x 32 bf16 (non-swap)
     uint64_t* full = reinterpret_cast<uint64_t*>(staging + (SWAP ? 0 : kStagingBytes));
     uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
+    uint64_t* sf_full = empty + STAGES;
+    uint64_t* acc_full = sf_full + STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
@@ -414,6 +431,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_full[s], 4);  // the four scale warps
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);
@@ -425,7 +443,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (prm.tma_store) prefetch_tmap(&tmap_y);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -434,6 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     int abort = 0;
 
+    if (warp < 8) setmaxnreg_dec<kLowRegs>();
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------------- producer
@@ -478,7 +497,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t phase = 0;
             int acc = 0;
             uint32_t acc_phase = 0;
-            uint32_t sfbuf = 0;
             WorkIter it(prm, blockIdx.x, gridDim.x);
             Work w;
             while (!abort && it.next(prm, w)) {
@@ -486,23 +504,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * Cfg::kAccStride;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
-                    // the TMA data of the stage is complete once the barrier phase flips; no
-                    // tcgen05 fence here (it would drain the MMA queue every K step)
                     if (!mbar_wait(&full[stage], phase, &abort)) break;
+                    if (!mbar_wait(&sf_full[stage], phase, &abort)) break;
+                    tc_fence_after();  // the scale warps' tcgen05.st precede these MMAs
                     const uint32_t sp = smem_u32(smem + stage * Cfg::kStageBytes);
                     const uint32_t sq = sp + Cfg::kPBytes;
-                    const uint32_t ssfp = sq + Cfg::kQBytes;
-                    const uint32_t ssfq = ssfp + Cfg::kSFPBytes;
-                    const uint32_t tsfp = tmem_base + Cfg::kSFBase + sfbuf * Cfg::kSFBufCols;
+                    const uint32_t tsfp = tmem_base + Cfg::kSFBase + stage * Cfg::kSFBufCols;
                     const uint32_t tsfq = tsfp + 8;
-                    sfbuf ^= 1u;
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        tc_cp_sf(tsfp + 4 * g, desc_sf(ssfp + 512 * g));
-#pragma unroll
-                        for (int i = 0; i < Cfg::kQBlocks; ++i)
-                            tc_cp_sf(tsfq + Cfg::kSFQColsPerGroup * g + 4 * i, desc_sf(ssfq + 1024 * i + 512 * g));
-                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t g = j >> 1;
@@ -512,7 +520,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tc_mma_mxf4(d_tmem, desc_sw128(sp + 32 * j), desc_sw128(sq + 32 * j),
                                     idesc | (id << 29) | (id << 4), sfa, sfb, (kt != w.k0 || j != 0) ? 1u : 0u);
                     }
-                    tc_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+                    tc_commit(&empty[stage]);  // frees the stage and its scale buffer once these MMAs have read them
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -526,13 +534,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------------ scale warps
+        // Warp (4 + sub) writes TMEM lanes 32 sub .. 32 sub + 31 of the stage's scale buffer,
+        // each lane 16 bytes of every atom (the bytes a 32x128b.warpx4 copy puts there):
+        // columns 0-7 the two P atoms, then per 4-block group g the Q atoms of each 128-row
+        // block, in the order of the MMA's scale addresses.  A stage is refilled only after
+        // the MMAs of its previous use completed, so its TMEM buffer is free once it is full.
+        constexpr int kVals = 2 + 2 * Cfg::kQBlocks;
+        const int sub = warp & 3;
+        int stage = 0;
+        uint32_t phase = 0;
+        WorkIter it(prm, blockIdx.x, gridDim.x);
+        Work w;
+        while (!abort && it.next(prm, w)) {
+            for (int kt = w.k0; kt < w.k1; ++kt) {
+                if (!mbar_wait(&full[stage], phase, &abort)) break;
+                const uint8_t* ssfp = smem + stage * Cfg::kStageBytes + Cfg::kPBytes + Cfg::kQBytes + lane * 16;
+                const uint8_t* ssfq = ssfp + Cfg::kSFPBytes;
+                uint4 v[kVals];
+                v[0] = *reinterpret_cast<const uint4*>(ssfp);
+                v[1] = *reinterpret_cast<const uint4*>(ssfp + 512);
+#pragma unroll
+                for (int g = 0; g < 2; ++g)
+#pragma unroll
+                    for (int i = 0; i < Cfg::kQBlocks; ++i)
+                        v[2 + g * Cfg::kQBlocks + i] = *reinterpret_cast<const uint4*>(ssfq + 1024 * i + 512 * g);
+                const uint32_t taddr =
+                    tmem_base + Cfg::kSFBase + stage * Cfg::kSFBufCols + (static_cast<uint32_t>(sub * 32) << 16);
+                tmem_st16(taddr, reinterpret_cast<const uint32_t*>(&v[0]));
+                if constexpr (kVals == 6) tmem_st8(taddr + 16, reinterpret_cast<const uint32_t*>(&v[4]));
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp >= 8) {
         // ------------------------------------------------------------------ epilogue
+        setmaxnreg_inc<kEpiRegs>();
         constexpr int kHalf = BN / 2;            // columns per epilogue warp
         constexpr int kChunk = kHalf >= 32 ? 32 : kHalf;
         const int sub = warp & 3;                // TMEM sub-partition this warp may read
-        const int half = (warp - 2) >> 2;        // which half of the tile's columns
-        const int etid = threadIdx.x - 64;       // 0..255 among the epilogue threads
+        const int half = (warp - 8) >> 2;        // which half of the tile's columns
+        const int etid = threadIdx.x - 256;      // 0..255 among the epilogue threads
         int acc = 0;
         uint32_t acc_phase = 0;
         WorkIter it(prm, blockIdx.x, gridDim.x);
@@ -568,7 +617,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             e.q0 = t.y_q + half * kHalf;
             e.p_end = t.p_end;
             e.q_end = t.q_end;
-            e.staging = staging + (warp - 2) * 2048;
+            e.staging = staging + (warp - 8) * 2048;
             finish_item<BN, SWAP>(prm, &tmap_y, w, e, v, abort);
         }
         if (lane == 0) bulk_wait_group<0>();  // output stores complete before the CTA exits
@@ -577,7 +626,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
 // ------------------------------------------------------------------ CTA-pair kernel
@@ -606,12 +655,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // epilogue's (setmaxnreg), which holds 128 accumulator columns per thread.
 // Scheduling (data-parallel waves then stream-K) works on pairs; partial-sum slots stay per CTA.
 constexpr int kPairStages = 5;
-constexpr int kPairThreads = 512;
-constexpr int kPairLaunchRegs = 65536 / kPairThreads;  // registers per thread at launch
-constexpr int kPairLowRegs = 80;                        // producer, MMA and scale warpgroups
-constexpr int kPairEpiRegs = 176;                       // epilogue warpgroups
-static_assert(2 * 128 * kPairLowRegs + 2 * 128 * kPairEpiRegs <= kPairThreads * kPairLaunchRegs,
-              "the register split must fit in the registers the block is launched with");
+constexpr int kPairThreads = kGemmThreads;  // same warp roles and register split
 struct PairCfg {
     static constexpr int kABytes = 128 * kStageKBytes;     // this CTA's 128 activation rows
     static constexpr int kBBytes = 128 * kStageKBytes;     // this CTA's 128 weight rows
@@ -677,7 +721,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     int abort = 0;
 
-    if (warp < 8) setmaxnreg_dec<kPairLowRegs>();
+    if (warp < 8) setmaxnreg_dec<kLowRegs>();
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------- producer (both CTAs)
@@ -794,7 +838,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
     } else if (warp >= 8) {
         // ----------------------------------------------------------- epilogue (both CTAs)
-        setmaxnreg_inc<kPairEpiRegs>();
+        setmaxnreg_inc<kEpiRegs>();
         constexpr int kHalf = BN / 2;
         const int sub = warp & 3;
         const int half = (warp - 8) >> 2;
@@ -895,7 +939,7 @@ static bool make_sf_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, i
 
 template <int BN, int STAGES, bool SWAP>
 static int smem_bytes() {
-    return STAGES * TileCfg<BN>::kStageBytes + (SWAP ? 0 : kStagingBytes) + (2 * STAGES + 4) * 8 + 16 + 1024;
+    return STAGES * TileCfg<BN>::kStageBytes + (SWAP ? 0 : kStagingBytes) + (3 * STAGES + 4) * 8 + 16 + 1024;
 }
 
 // Tensor map of the bf16 output [rows][cols]: 32 x 32 boxes, 64-byte swizzle.
@@ -910,6 +954,12 @@ static bool make_out_map(CUtensorMap* map, void* y, int64_t rows, int64_t cols, 
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// setmaxnreg.inc takes registers from those the block was launched with: a kernel built with
+// fewer than the split assumes would wait forever there, so it is never launched.
+static bool register_split_fits(const cudaFuncAttributes& fa) {
+    return fa.numRegs * kGemmThreads >= 2 * 128 * kLowRegs + 2 * 128 * kEpiRegs;
 }
 
 // Per-device cache of a launch-configuration query (the answers depend only on the device).
@@ -938,13 +988,18 @@ template <int BN, int STAGES, bool SWAP>
 static int grid_ctas_query() {
     auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP>;
     const int smem = smem_bytes<BN, STAGES, SWAP>();
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || !register_split_fits(fa)) {
+        cudaGetLastError();
+        return -1;
+    }
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
     // all of the unified L1/shared storage as shared memory, so small configurations fit twice per SM
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return -1;
     int occ = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kGemmThreads, smem) != cudaSuccess || occ < 1)
         occ = 1;
-    if (occ * TileCfg<BN>::kTmemCols > 512) occ = 512 / TileCfg<BN>::kTmemCols;
+    if (occ * TileTmem<BN, STAGES>::kCols > 512) occ = 512 / TileTmem<BN, STAGES>::kCols;
     return sm_count() * occ;  // occ is 1: the runtime keeps tensor-memory kernels at one CTA per SM
 }
 
@@ -1026,6 +1081,11 @@ static bool kernel_attributes() {
     return cached_per_device(cache, [] {
                auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP, GROUPED>;
                const int smem = smem_bytes<BN, STAGES, SWAP>();
+               cudaFuncAttributes fa;
+               if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || !register_split_fits(fa)) {
+                   cudaGetLastError();
+                   return -1;
+               }
                return (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
                        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) == cudaSuccess)
                           ? 1
@@ -1129,7 +1189,7 @@ static int gemm_pairs_query() {
         cudaGetLastError();
         return 0;
     }
-    if (fa.numRegs * kPairThreads < 2 * 128 * kPairLowRegs + 2 * 128 * kPairEpiRegs) return 0;
+    if (!register_split_fits(fa)) return 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) != cudaSuccess) return 0;
     cudaLaunchConfig_t cfg = {};

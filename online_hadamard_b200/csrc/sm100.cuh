@@ -1,6 +1,6 @@
 // sm100.cuh -- thin inline-PTX wrappers for the Blackwell (sm_100a) features the kernels
 // use: mbarriers with bounded waits, TMA tensor and bulk copies, tcgen05 tensor-memory
-// allocation, copies, block-scaled MMA, commits and loads.  Each wrapper is one PTX
+// allocation, block-scaled MMA, commits, loads and stores.  Each wrapper is one PTX
 // instruction (or a short fixed sequence) written from the PTX ISA's instruction forms.
 #pragma once
 
@@ -157,23 +157,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Descriptor of a 32-row x 16-byte scale-factor block, rows contiguous (no swizzle):
-// 8-row core matrices 128 B apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-    d |= static_cast<uint64_t>(128 >> 4) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    return d;
-}
-
-// Copy 32 rows x 128 bits from shared memory into TMEM columns [taddr, taddr+4) of
-// lanes 0-31, replicated into the other three 32-lane sub-partitions.
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
 // D (+)= (A * 2^sfA) (B * 2^sfB)^T for one K = 64 slice of MXFP4 operands.
 __device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
@@ -321,11 +304,6 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 }
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Scale-factor copy into the same TMEM columns of both CTAs, each from its own shared memory.
-__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Pair MMA (M = 256 over the two CTAs): D (+)= (A * 2^sfA) (B * 2^sfB)^T for K = 64.
