@@ -10,7 +10,7 @@
 // Activations", Abstract: per-channel scale + block-Hadamard online on the activations,
 // inverse transforms absorbed into the weights, MXFP4 W4A4, round-to-nearest weights.
 //
-// Work split: one thread owns one 32-element block column and walks a group of rows, so
+// Work split (large inputs): one thread owns one 32-element block column and walks a group of rows, so
 // its 32 multipliers stay in registers and the whole 32-point butterfly runs in its
 // registers with no cross-lane traffic.  A warp covers 32 consecutive blocks (2 KB of
 // bf16) of one row: its four 16-byte loads per row touch every sector of that span, and
@@ -19,6 +19,12 @@
 // intrinsic (scalar or the sm_100 packed f32x2 form), so the scale cannot be contracted
 // into the first butterfly and the result is bit-identical to the canonical sequential
 // order.  The kernel is HBM-bound: 2 (or 4) bytes in, 0.53 bytes out per element.
+//
+// Small activation inputs (decode, short prefill) are bound by latency instead: few threads,
+// each with a long serial chain of loads and transform arithmetic.  There the transform runs
+// with two threads per block (mx_quant_half_kernel below): half the registers and half the
+// serial work per thread, twice the threads in flight.  Its extra shuffles make it slower
+// once the input fills the GPU, so the launch picks the kernel by input size.
 #include <cstdint>
 #include <cmath>
 #include <vector>
@@ -282,9 +288,146 @@ static unsigned quant_blocks(int64_t R, int64_t K, int64_t rpg) {
     return static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
 }
 
+
+// ---------------------------------------------------------------- half-block transform
+//
+// Two adjacent lanes per 32-element block: each loads, scales and transforms 16 elements,
+// stages h = 1, 2, 4, 8 in its own registers.  The last stage (h = 16) pairs element i of the
+// low half with element i of the high half, so the two lanes swap their 16 values once and
+// the low lane keeps the sums, the high lane the differences -- the same fp32 operations in
+// the same order as the whole-block butterfly, so the codes are bit-identical.  amax is the
+// larger of the two halves' maxima; each lane converts and stores its 8 code bytes, the low
+// lane the scale byte.
+__device__ __forceinline__ void half_scale_fwht(float2 (&u)[8], const float2 (&m)[8], int hf, unsigned pair_mask) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) u[p] = __fmul2_rn(u[p], m[p]);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {  // h = 1: the two halves of a pair
+        const float a = u[p].x, b = u[p].y;
+        u[p] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int hp = 1; hp < 8; hp <<= 1) {  // h = 2, 4, 8: whole pairs, packed
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            if ((p & hp) == 0) {
+                const float2 a = u[p], b = u[p + hp];
+                u[p] = __fadd2_rn(a, b);
+                u[p + hp] = fsub2_rn(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {  // h = 16 across the lane pair: a = low lane's value, b = high's
+        float2 o;
+        o.x = __shfl_xor_sync(pair_mask, u[p].x, 1);
+        o.y = __shfl_xor_sync(pair_mask, u[p].y, 1);
+        u[p] = hf == 0 ? __fadd2_rn(u[p], o) : fsub2_rn(o, u[p]);
+    }
+}
+
+__device__ __forceinline__ void half_block(const uint4 (&raw)[2], const float2 (&m)[8], int hf, unsigned pair_mask,
+                                           uint8_t* codes8, uint8_t* scale_byte) {
+    float2 u[8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)  // bf16 -> fp32 is exact: the bits move up 16 places
+            u[4 * j + t] = make_float2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xFFFF0000u));
+    }
+    half_scale_fwht(u, m, hf, pair_mask);
+    const float* f = reinterpret_cast<const float*>(u);
+    float amax = fmax3(fabsf(f[0]), fabsf(f[1]), fabsf(f[2]));
+#pragma unroll
+    for (int i = 3; i + 1 < 16; i += 2) amax = fmax3(amax, fabsf(f[i]), fabsf(f[i + 1]));
+    amax = fmaxf(amax, fabsf(f[15]));
+    amax = fmaxf(amax, __shfl_xor_sync(pair_mask, amax, 1));
+    const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
+    const uint32_t e = E >= 3u ? E - 2u : 0u;
+    const float inv = __uint_as_float((254u - e) << 23);  // 2^(127 - e), a normal float
+    const float2 inv2 = make_float2(inv, inv);
+    const uint32_t c0 = cvt_e2m1x8(__fmul2_rn(u[0], inv2), __fmul2_rn(u[1], inv2), __fmul2_rn(u[2], inv2),
+                                   __fmul2_rn(u[3], inv2));
+    const uint32_t c1 = cvt_e2m1x8(__fmul2_rn(u[4], inv2), __fmul2_rn(u[5], inv2), __fmul2_rn(u[6], inv2),
+                                   __fmul2_rn(u[7], inv2));
+    *reinterpret_cast<uint2*>(codes8) = make_uint2(c0, c1);
+    if (hf == 0) *scale_byte = static_cast<uint8_t>(e);
+}
+
+constexpr int kHalfThreads = 128;
+constexpr int kHalfMinBlocks = 6;                        // 80 registers: six CTAs per SM
+constexpr int64_t kHalfKernelMaxElems = int64_t(1) << 22;  // above this the whole-block kernel wins
+
+// Thread = (run of `rpg` rows) x (block column kb) x (half hf), halves fastest, then columns;
+// the low half of a padded block column (kb >= K/32) writes the zero scale bytes of its rows.
+__global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_kernel(
+    const uint16_t* __restrict__ x, int64_t R, int64_t K, int64_t rpg, const float* __restrict__ mult,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    griddep_launch_dependents();
+    const int64_t kb_real = K / 32;
+    const int64_t kbp = padded_blocks(K);
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * kHalfThreads + threadIdx.x;
+    const int hf = static_cast<int>(item & 1);
+    const int64_t kb = (item >> 1) % kbp;
+    const int64_t r0 = ((item >> 1) / kbp) * rpg;
+    if (r0 >= R) return;  // both lanes of a pair leave together: same block column, same rows
+    const int64_t n = r0 + rpg < R ? rpg : R - r0;
+    if (kb >= kb_real) {
+        if (hf == 0)
+            for (int64_t r = r0; r < r0 + n; ++r) scales[scale_offset(r, kb, kbp)] = 0;
+        return;
+    }
+    const unsigned pair_mask = 3u << (threadIdx.x & 30u);
+    const int64_t k0 = kb * 32 + hf * 16;
+    float2 m[8];
+    const float4* mp = reinterpret_cast<const float4*>(mult + k0);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 t = __ldg(mp + j);
+        m[2 * j] = make_float2(t.x, t.y);
+        m[2 * j + 1] = make_float2(t.z, t.w);
+    }
+    auto load = [&](int64_t r, uint4 (&b)[2]) {
+        const uint4* p = reinterpret_cast<const uint4*>(x + r * K + k0);
+        b[0] = __ldcs(p);
+        b[1] = __ldcs(p + 1);
+    };
+    auto out = [&](int64_t r) { return codes + r * (K / 2) + kb * 16 + hf * 8; };
+    int64_t i = 0;
+    for (; i + 1 < n; i += 2) {  // two rows at a time, both loaded before either is used
+        uint4 b0[2], b1[2];
+        load(r0 + i, b0);
+        load(r0 + i + 1, b1);
+        half_block(b0, m, hf, pair_mask, out(r0 + i), scales + scale_offset(r0 + i, kb, kbp));
+        half_block(b1, m, hf, pair_mask, out(r0 + i + 1), scales + scale_offset(r0 + i + 1, kb, kbp));
+    }
+    if (i < n) {
+        uint4 b0[2];
+        load(r0 + i, b0);
+        half_block(b0, m, hf, pair_mask, out(r0 + i), scales + scale_offset(r0 + i, kb, kbp));
+    }
+}
+
+// Rows per thread of the half-block kernel: enough threads for one resident wave (six CTAs of
+// 128 per SM), rows walked by each otherwise.
+static int64_t half_rows_per_thread(int64_t R, int64_t K) {
+    const int64_t items = 2 * padded_blocks(K);
+    const int64_t target = static_cast<int64_t>(sm_count()) * kHalfMinBlocks * kHalfThreads;
+    const int64_t rpg = (R * items + target - 1) / target;
+    return rpg < 1 ? 1 : rpg;
+}
+
 // Launch helpers used by the C entry points and by the linear.
 int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const float* act_mult,
                                uint8_t* Aq, uint8_t* As, cudaStream_t stream) {
+    if (M * K <= kHalfKernelMaxElems) {
+        const int64_t rpg = half_rows_per_thread(M, K);
+        const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
+        mx_quant_half_kernel<<<static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads), kHalfThreads, 0,
+                               stream>>>(x, M, K, rpg, act_mult, Aq, As);
+        return launch_status();
+    }
     const int64_t rpg = quant_rows_per_thread(M, K);
     mx_quant_kernel<QuantMode::kActTransform><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
         x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq, As);
