@@ -892,19 +892,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
 // --------------------------------------------------------------------------- host side
 
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 // Tensor map of an MXFP4 code matrix [rows][K/2] bytes: boxes of box_rows x 128 bytes,
 // 128-byte swizzle, zero fill past the edges (ragged M, N and K tails).
 static bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {

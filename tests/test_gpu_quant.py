@@ -52,6 +52,28 @@ def test_act_transform_quant_matches_oracle(mq, wl):
     print(wl.name, wl.M, stats)
 
 
+@pytest.mark.parametrize("M,K", [(1037, 4128), (4099, 1056), (64, 65600)], ids=lambda v: str(v))
+def test_act_quant_large_ragged(mq, M, K):
+    """Inputs above the small-input size, so the shared-memory-fed kernel runs, with rows that
+    do not fill its 32-row tiles and K that does not fill its 256-element strips (padded scale
+    blocks): transform and plain codes against the oracle."""
+    assert M * K > (1 << 22)
+    rng = np.random.default_rng(M + K)
+    xf32 = rng.standard_t(4, (M, K)).astype(np.float32) * rng.uniform(0.1, 30.0, (1, K)).astype(np.float32)
+    xb = torch.from_numpy(xf32).to(torch.bfloat16)
+    s = rng.uniform(0.05, 5.0, K).astype(np.float32)
+    a, _ = oracle.multipliers(s)
+    Aq, As = mq.macaq_act_transform_quant(xb.cuda(), torch.from_numpy(a).cuda())
+    Pq, Ps = mq.macaq_act_quant_plain(xb.cuda())
+    torch.cuda.synchronize()
+    xf = xb.float().numpy()
+    V = oracle.transform_f32(xf, a)
+    rc, rs = oracle.quantize_mx(V)
+    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, M, K, V)
+    pc, ps = oracle.quantize_mx(xf)
+    gu.compare_mx(gu.to_np(Pq), gu.to_np(Ps), pc, ps, M, K, xf)
+
+
 @pytest.mark.parametrize("wl", [wls.TINY, wls.LLAMA_UP, wls.QWEN_DOWN], ids=lambda w: w.name)
 def test_act_quant_plain_matches_oracle(mq, wl):
     x = wls.make_x(wl)
