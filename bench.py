@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import statistics
 import json
 import math
 import os
@@ -313,12 +314,18 @@ def time_eager(fn, steps, warmup, device):
     return e0.elapsed_time(e1) / steps
 
 
-def time_loop(fn, steps, warmup, device):
-    """ms per call of fn, from a graph-captured loop of `steps` calls."""
-    g = GraphLoop(fn, steps, warmup, device)
-    ms = g.time_ms() / steps
-    del g
-    return ms
+def time_ab(fns, steps, warmup, device, rounds=5):
+    """ms per call of each fn in `fns` (name -> fn), each captured as a graph of `steps` calls;
+    the graphs are replayed in turn for `rounds` rounds and each fn's median is returned, so a
+    drift of the clock or of the board's power state during the run falls on every fn alike
+    (the comparisons -- overhead against plain MXFP4 -- are differences of a few percent)."""
+    loops = {name: GraphLoop(fn, steps, warmup, device) for name, fn in fns.items()}
+    times = {name: [] for name in fns}
+    for _ in range(rounds):
+        for name, g in loops.items():
+            times[name].append(g.time_ms() / steps)
+    del loops
+    return {name: statistics.median(v) for name, v in times.items()}
 
 
 # --------------------------------------------------------------------------- CPU baseline
@@ -432,15 +439,27 @@ def main():
     torch.cuda.synchronize(device)
     barrier()
     torch.cuda.synchronize(device)
+    # the timed replay lasts milliseconds, shorter than nvidia-smi's sampling period: keep the
+    # same graph replaying (untimed) for ~0.4 s so the clock samples are taken under this load
+    t_soak = time.perf_counter()
+    soak = 0
+    while time.perf_counter() - t_soak < 0.4:
+        loop.graph.replay()
+        soak += 1
+        if soak % 8 == 0:
+            torch.cuda.synchronize(device)
+    torch.cuda.synchronize(device)
     clk = clocks.stop()
+    clk["window"] = f"the timed replay and {soak} untimed replays of the same graph right after it"
     del loop
     ms = max_over_ranks(ms_total / args.steps)
     value = whole_job_tflops(world, wl.flops, ms)
 
-    # ---- dominant kernel, the comparators and end to end (same rotation)
-    ms_gemm = time_loop(layer.gemm, args.steps, args.warmup, device)
-    ms_plain = time_loop(layer.plain, args.steps, args.warmup, device)
-    ms_xform = time_loop(layer.transform_only, args.steps, args.warmup, device)
+    # ---- dominant kernel, the comparators and end to end (same rotation); the overhead
+    # compares medians of alternating replays of the W4A4 and plain-MXFP4 linears
+    ab = time_ab({"linear": layer.linear, "plain": layer.plain, "gemm": layer.gemm,
+                  "transform": layer.transform_only}, args.steps, args.warmup, device)
+    ms_gemm, ms_plain, ms_xform, ms_lin_ab = ab["gemm"], ab["plain"], ab["transform"], ab["linear"]
     e2e_steps = max(3, min(args.steps, 10))
     ms_e2e = max_over_ranks(time_eager(layer.e2e, e2e_steps, 3, device))
     gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
@@ -470,9 +489,10 @@ def main():
                          "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
                          "ms_per_launch": ms_gemm},
             "linear_roofline": linear_roofline(wl, ms, fp4_peak, peaks["hbm_gbs"]),
-            "overhead": {"linear_ms": ms, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
-                         "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
-                         "vs_gemm_only_pct": 100.0 * (ms / ms_gemm - 1.0),
+            "overhead": {"linear_ms": ms_lin_ab, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
+                         "vs_plain_mxfp4_pct": 100.0 * (ms_lin_ab / ms_plain - 1.0),
+                         "vs_gemm_only_pct": 100.0 * (ms_lin_ab / ms_gemm - 1.0),
+                         "method": "medians of 5 alternating graph replays per variant",
                          "transform_quant_ms": ms_xform,
                          "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
             "e2e": {"value": whole_job_tflops(world, wl.flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
@@ -542,8 +562,8 @@ def stack_sweep(mq, device, peaks, Ms=(1, 32, 512, 4096), steps=3, warmup=2):
             for K, N, Wq, Ws, am in lin:
                 mq.macaq_mxfp4_linear(xs[K], Wq, Ws, N, y=ys[N], workspace=ws)
 
-        ms = time_loop(w4a4, steps, warmup, device)
-        ms_plain = time_loop(plain, steps, warmup, device)
+        ab = time_ab({"w4a4": w4a4, "plain": plain}, steps, warmup, device, rounds=3)
+        ms, ms_plain = ab["w4a4"], ab["plain"]
         flops = sum(2.0 * M * K * N for K, N, *_ in lin)
         nbytes = sum(wls.alg_bytes(wls.Workload("", 5, M, K, N, "normal", 0.0, 1.0)) for K, N, *_ in lin)
         t_roof = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
@@ -584,10 +604,11 @@ def moe_sweep(mq, device, peaks, token_counts=(16, 4096), steps=10, warmup=3):
                                                layer=E * li + E), rows, device)
             y = torch.empty(rows, N, dtype=torch.bfloat16, device=device)
             ws = torch.empty(max(mq.grouped_workspace_bytes(counts, N, K), 1), dtype=torch.uint8, device=device)
-            ms = time_loop(lambda i: mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N, y=y, workspace=ws),
-                           steps, warmup, device)
-            ms_plain = time_loop(lambda i: mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N, y=y, workspace=ws),
-                                 steps, warmup, device)
+            ab = time_ab({"w4a4": lambda i: mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N, y=y, workspace=ws),
+                          "plain": lambda i: mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N, y=y,
+                                                                          workspace=ws)},
+                         steps, warmup, device)
+            ms, ms_plain = ab["w4a4"], ab["plain"]
             active = sum(1 for c in counts if c)
             flops = 2.0 * rows * K * N
             nbytes = active * N * K * (0.5 + 1 / 32) + 2.0 * rows * (K + N) + 4.0 * K * active
@@ -610,8 +631,8 @@ def secondary(mq, device, peaks, args):
     for M in wls.QWEN_DECODE_M:
         wl = wls.QWEN_UP_DECODE.with_m(M)
         layer = Layer(mq, wl, device)
-        ms = time_loop(layer.linear, steps, args.warmup, device)
-        ms_plain = time_loop(layer.plain, steps, args.warmup, device)
+        ab = time_ab({"linear": layer.linear, "plain": layer.plain}, steps, args.warmup, device)
+        ms, ms_plain = ab["linear"], ab["plain"]
         res[f"{wl.name}_M{M}"] = {"ms": ms, "gbs": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9,
                                    "frac_hbm": wls.alg_bytes(wl) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                    "linear_roofline": linear_roofline(wl, ms, peaks["bf16_tflops"] * FP4_OVER_BF16,
@@ -621,9 +642,8 @@ def secondary(mq, device, peaks, args):
         torch.cuda.empty_cache()
     wl = wls.QWEN_DOWN
     layer = Layer(mq, wl, device, copies=2)
-    ms = time_loop(layer.linear, steps, args.warmup, device)
-    ms_plain = time_loop(layer.plain, steps, args.warmup, device)
-    ms_gemm = time_loop(layer.gemm, steps, args.warmup, device)
+    ab = time_ab({"linear": layer.linear, "plain": layer.plain, "gemm": layer.gemm}, steps, args.warmup, device)
+    ms, ms_plain, ms_gemm = ab["linear"], ab["plain"], ab["gemm"]
     t = wl.flops / (ms * 1e-3) / 1e12
     res[wl.name] = {"ms": ms, "tflops": t, "frac_fp4_peak": t / (peaks["bf16_tflops"] * FP4_OVER_BF16),
                     "linear_roofline": linear_roofline(wl, ms, peaks["bf16_tflops"] * FP4_OVER_BF16, peaks["hbm_gbs"]),
