@@ -83,7 +83,8 @@ int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
 /* Bytes of scratch macaq_mxfp4_gemm uses for its stream-K schedule on the current device
  * (256 eight-byte flag words and a 128-row fp32 partial-sum slot per CTA of the persistent
  * grid; depends on M and the device's SM count).  The scratch needs no initialisation: a
- * flag word counts as written only when it holds the tag of the current launch. */
+ * flag word counts as written only when it holds the tag of the current launch, and the
+ * launch clears the words it consumed, so calls captured in a CUDA graph may be replayed. */
 size_t macaq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Bytes of scratch macaq_w4a4_linear (and macaq_mxfp4_linear) needs on the current device:

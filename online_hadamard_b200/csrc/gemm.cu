@@ -271,8 +271,9 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
     if (w.kind == kPartial) {
         // fp32 partial to this CTA's slot, [chunk of 4 columns][epilogue thread]; then this
         // thread's flag word takes the launch's tag (release: after its part of the partial).
-        // The owner's thread with the same index reads exactly this part, so no flag is
-        // ever shared, counted or cleared.
+        // The owner's thread with the same index reads exactly this part and then clears the
+        // word, so no flag is shared or counted, and every launch starts from cleared words
+        // (a CUDA graph replays a captured launch with the same tag).
         float4* slot = reinterpret_cast<float4*>(prm.partials + static_cast<int64_t>(e.slot_self) * (kBM * BN));
 #pragma unroll
         for (int j = 0; j < kHalf / 4; ++j)
@@ -287,9 +288,9 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
         for (int c = e.unit + 1; c <= w.c_last; ++c) {
             if (U * c / G == U * (c + 1) / G) continue;  // empty range: no partial
             const int slot_id = c * e.slot_stride + e.slot_off;
+            uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + e.etid;
             if (!abort) {
                 const long long t0 = clock64();
-                const uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + e.etid;
                 while (ld_acquire64(flag) != prm.tag) {
                     if (clock64() - t0 > kWaitLimitCycles) {
                         atomicExch(&g_device_status, MACAQ_ETIMEOUT);
@@ -307,6 +308,9 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
                 v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q.z);
                 v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q.w);
             }
+            // consumed: clear the word, so a later launch that repeats this tag (a graph replay)
+            // cannot take it for its own contributor's signal
+            __stcg(reinterpret_cast<unsigned long long*>(flag), 0ull);
         }
     }
     if constexpr (!SWAP && kHalf % 32 == 0) {
@@ -1026,8 +1030,9 @@ static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch
 }
 
 // Stream-K scratch: a flag word per (CTA slot, epilogue thread), then one 128 x BN fp32
-// partial-sum slot per CTA.  Flags hold the tag of the launch that last wrote them, so the
-// scratch needs no clearing: any contents on entry are fine.
+// partial-sum slot per CTA.  A flag counts as set only when it holds the tag of the current
+// launch, and the owner clears every flag it consumed, so the scratch needs no initialisation
+// (any contents on entry are fine) and a CUDA graph may replay a captured launch, tag included.
 static size_t streamk_flag_bytes(int ctas) {
     return (static_cast<size_t>(ctas) * kEpiThreads * 8 + 255) / 256 * 256;
 }

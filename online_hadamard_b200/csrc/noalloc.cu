@@ -19,8 +19,8 @@
 //     runs its data-parallel schedule (same results up to fp32 summation order);
 //   * every call shares it and it keeps the previous call's contents.  Nothing in it has
 //     to start at zero: each call writes every code byte and every scale byte of its real
-//     rows before reading them, the stream-K flags only ever match the tag of the launch
-//     that wrote them, and the bytes it does not write (padded rows of the last 128-row scale atom, stale
+//     rows before reading them, a stream-K flag counts only when it holds the tag of the
+//     current launch (and each launch clears the flags it consumed), and the bytes it does not write (padded rows of the last 128-row scale atom, stale
 //     partial sums) are never used for a stored output;
 //   * two calls whose kernels overlap on the GPU (different streams without ordering, or
 //     several host threads) race on the array and corrupt each other's results: order

@@ -98,6 +98,41 @@ def test_streamk_workspace_reused_and_dirty(mq, M, N, K):
     assert gu.rel_fro(gu.to_np(ys[0]), oracle.mx_gemm(Ac, As, Wc, Ws)) <= TOL
 
 
+@pytest.mark.parametrize("M,N,K", [(16, 2048, 8192), (300, 2048, 16384)], ids=lambda v: str(v))
+def test_streamk_graph_replays_with_new_inputs(mq, M, N, K):
+    """A stream-K GEMM captured in a CUDA graph is replayed with the same launch tag every
+    time; each replay here gets new operand codes (copied into the captured buffers) and must
+    give exactly what an eager call on those codes gives, i.e. no owner may take a flag left
+    set by the previous replay for its own contributor's signal."""
+    rng = np.random.default_rng(7 * M + K)
+    inputs = []
+    for _ in range(4):
+        Ac, As = random_mx(rng, M, K)
+        Wc, Ws = random_mx(rng, N, K)
+        inputs.append((*to_device_mx(Ac, As, M, K), *to_device_mx(Wc, Ws, N, K)))
+    bufs = [t.clone() for t in inputs[0]]
+    ws = torch.empty(mq.gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    expect = [mq.macaq_mxfp4_gemm(*inp, M, N, K, out_fp32=True, workspace=ws).clone() for inp in inputs]
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        mq.macaq_mxfp4_gemm(*bufs, M, N, K, y=y, out_fp32=True, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mq.macaq_mxfp4_gemm(*bufs, M, N, K, y=y, out_fp32=True, workspace=ws)
+    for r in range(8):
+        for dst, src in zip(bufs, inputs[r % 4]):
+            dst.copy_(src)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, expect[r % 4]), f"replay {r} differs from the eager result"
+    assert mq.macaq_device_status() == 0
+
+
 def test_gemm_exact_small_integers(mq):
     # all elements in {0, +-0.5, +-1} and scale 127: every partial sum is exact in fp32
     rng = np.random.default_rng(5)
