@@ -1000,8 +1000,12 @@ static int grid_ctas_query() {
 // scheduling units (CTAs, or CTA pairs), chosen by its estimated critical path in K steps:
 //   data-parallel  ceil(tiles / units) rounds of whole tiles;
 //   stream-K       all but the last full wave data-parallel, the K steps of the rest split
-//                  evenly over every unit, plus the fix-up's cost `streamk_cost` (needs the
-//                  stream-K scratch).
+//                  evenly over the units, plus the fix-up's cost `streamk_cost` (needs the
+//                  stream-K scratch).  Each unit takes at least a quarter of a tile's K steps,
+//                  so a tile has at most four contributors besides its owner: the owner waits
+//                  for and reads their partials one after another, and a tile split eighteen
+//                  ways (a 1024-row weight matrix at decode spread over 148 CTAs) took 19.5 us
+//                  where its 2.8 MB of weights stream in well under one.
 // (Splitting only the leftover tiles, each over a few units, measured slower on B200: the
 // owner reads its contributors' partials one after another.)
 struct Schedule {
@@ -1015,13 +1019,17 @@ static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch
     const int64_t full = tiles / units, rem = tiles % units;
     const int64_t est_dp = (full + (rem ? 1 : 0)) * KT;
     const int64_t dp = (full > 0 ? full - 1 : 0) * units;
-    const int64_t est_sk = (dp / units) * KT + ((tiles - dp) * KT + units - 1) / units + streamk_cost;
+    const int64_t sk_units = (tiles - dp) * static_cast<int64_t>(KT);
+    const int64_t min_steps = (KT + 3) / 4;  // per splitting unit: at most four contributors per tile
+    int64_t split = (sk_units + min_steps - 1) / min_steps;
+    if (split > units) split = units;
+    const int64_t est_sk = (dp / units) * KT + (sk_units + split - 1) / split + streamk_cost;
     Schedule s;
     if (scratch && rem != 0 && KT > 1 && est_sk <= est_dp) {
         s.dp_tiles = static_cast<int>(dp);
-        s.sk_units = (tiles - dp) * static_cast<int64_t>(KT);
-        s.grid = units < s.sk_units ? units : s.sk_units;  // every unit gets at least one K step
-        s.sk_count = static_cast<int>(s.grid);              // the K steps go to the units launched
+        s.sk_units = sk_units;
+        s.sk_count = static_cast<int>(split);  // units 0 .. split-1 share the K steps
+        s.grid = dp > 0 ? units : split;        // all units when whole tiles precede the split
     } else {
         s.dp_tiles = static_cast<int>(tiles);
         s.grid = units < tiles ? units : tiles;
