@@ -1001,11 +1001,13 @@ static int grid_ctas_query() {
 //   data-parallel  ceil(tiles / units) rounds of whole tiles;
 //   stream-K       all but the last full wave data-parallel, the K steps of the rest split
 //                  evenly over the units, plus the fix-up's cost `streamk_cost` (needs the
-//                  stream-K scratch).  Each unit takes at least a quarter of a tile's K steps,
-//                  so a tile has at most four contributors besides its owner: the owner waits
-//                  for and reads their partials one after another, and a tile split eighteen
-//                  ways (a 1024-row weight matrix at decode spread over 148 CTAs) took 19.5 us
-//                  where its 2.8 MB of weights stream in well under one.
+//                  stream-K scratch).  A tile is split at most in two when it is short (<= 32
+//                  K steps), else in pieces of at least 16 K steps and at most four: the owner
+//                  waits for and reads its contributors' partials one after another, and each
+//                  one measured 1-2.5 us (a 1024-row weight matrix at decode, split eighteen
+//                  ways over 148 CTAs, took 19.5 us for 2.8 MB of weights; in two, 8.3 us),
+//                  while long tiles need all SMs streaming (the 25600-deep decode down
+//                  projection in two pieces: 23.0 us on 80 CTAs against 20.2 us on 148).
 // (Splitting only the leftover tiles, each over a few units, measured slower on B200: the
 // owner reads its contributors' partials one after another.)
 struct Schedule {
@@ -1020,7 +1022,8 @@ static Schedule plan_schedule(int64_t tiles, int64_t units, int KT, bool scratch
     const int64_t est_dp = (full + (rem ? 1 : 0)) * KT;
     const int64_t dp = (full > 0 ? full - 1 : 0) * units;
     const int64_t sk_units = (tiles - dp) * static_cast<int64_t>(KT);
-    const int64_t min_steps = (KT + 3) / 4;  // per splitting unit: at most four contributors per tile
+    const int64_t half = (KT + 1) / 2, quarter = (KT + 3) / 4;
+    const int64_t min_steps = half < (quarter > 16 ? quarter : 16) ? half : (quarter > 16 ? quarter : 16);
     int64_t split = (sk_units + min_steps - 1) / min_steps;
     if (split > units) split = units;
     const int64_t est_sk = (dp / units) * KT + (sk_units + split - 1) / split + streamk_cost;

@@ -48,9 +48,10 @@ SHAPES = [
     (1, 256, 256), (1, 7, 32), (4, 136, 96), (16, 384, 512), (17, 200, 288), (33, 520, 800),
     (64, 256, 1024), (65, 130, 256), (100, 1000, 800), (128, 128, 256), (129, 300, 320),
     (256, 512, 512), (300, 520, 1056), (511, 777, 640), (1024, 2048, 2048),
-    # long K, few tiles: stream-K splits every tile across many CTAs (owner + ~10-18
-    # contributors), swap-AB and CTA-pair kernels (1280 x 2048: 40 tiles on 74 pairs)
-    (16, 2048, 8192), (200, 1024, 8192), (70, 1100, 6144), (1280, 2048, 16384),
+    # long K, few tiles: stream-K splits tiles between CTAs (owner + 1 contributor for
+    # tiles of <= 32 K steps, up to 3 for longer ones), swap-AB and CTA-pair kernels
+    # (1280 x 2048: 40 tiles on 74 pairs)
+    (16, 2048, 8192), (200, 1024, 8192), (70, 1100, 6144), (16, 1024, 16384), (1280, 2048, 16384),
 ]
 
 
