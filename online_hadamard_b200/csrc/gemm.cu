@@ -647,8 +647,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //     stage's TMEM scale buffer with tcgen05.st, in the layout a 32x128b.warpx4 copy gives
 //     (each lane's four columns hold 16 bytes of an atom, repeated in every sub-partition),
 //     and arrive on the even CTA's "sf_full" barrier.  Issuing the copies as tcgen05.cp from
-//     the MMA thread instead puts six copies per K step into the MMA issue stream, about a
-//     third of the mainloop on these shapes;
+//     the MMA thread instead puts six copies per K step into the MMA issue stream (measured:
+//     64.4 us against 53 us for the Llama-3-8B up projection, 2048 x 4096 x 14336);
 //   - the even CTA's single MMA thread waits for both barriers, issues the pair MMAs and
 //     multicasts each stage's release to both CTAs' "empty" barriers (which also free the
 //     stage's TMEM scale buffer) and each tile's completion to both "acc_full" barriers;
