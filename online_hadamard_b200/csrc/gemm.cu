@@ -261,6 +261,41 @@ struct EpiCtx {
     uint8_t* staging;             // this warp's 2 KB output staging buffer (TMA-store path)
 };
 
+// Owner of a split tile: waits (bounded) for each contributor's flag, adds its partial sums to
+// `sum` (this thread's BN/2 columns, contributors in order) and clears the flag, so a later
+// launch repeating this launch's tag (a CUDA graph replay) cannot take it for its own signal.
+template <int BN>
+__device__ __forceinline__ void sum_partials(const GemmParams& prm, const Work& w, int unit, int slot_stride,
+                                             int slot_off, int etid, float* sum, int& abort) {
+    constexpr int kHalf = BN / 2;
+    const int64_t U = prm.sk_units, G = prm.sk_count;
+    for (int c = unit + 1; c <= w.c_last; ++c) {
+        if (U * c / G == U * (c + 1) / G) continue;  // empty range: no partial
+        const int slot_id = c * slot_stride + slot_off;
+        uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + etid;
+        if (!abort) {
+            const long long t0 = clock64();
+            while (ld_acquire64(flag) != prm.tag) {
+                if (clock64() - t0 > kWaitLimitCycles) {
+                    atomicExch(&g_device_status, MACAQ_ETIMEOUT);
+                    abort = 1;
+                    break;
+                }
+            }
+        }
+        const float4* slot = reinterpret_cast<const float4*>(prm.partials + static_cast<int64_t>(slot_id) * (kBM * BN));
+#pragma unroll
+        for (int j = 0; j < kHalf / 4; ++j) {
+            const float4 q = __ldcg(slot + j * kEpiThreads + etid);
+            sum[4 * j] += q.x;
+            sum[4 * j + 1] += q.y;
+            sum[4 * j + 2] += q.z;
+            sum[4 * j + 3] += q.w;
+        }
+        __stcg(reinterpret_cast<unsigned long long*>(flag), 0ull);
+    }
+}
+
 // After the accumulator of `w` is in registers (v = this thread's BN/2 fp32 columns): write a
 // stream-K partial, or add the contributors' partials (owner), then store y.
 template <int BN, bool SWAP>
@@ -592,6 +627,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         Work w;
         while (!abort && it.next(prm, w)) {
             const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, gt, w.tile);
+            // Narrow tiles (decode): the owner of a split tile adds its contributors' partial
+            // sums while its own MMAs still run.  The contributors did their part of the tile
+            // first in their ranges; the owner reaches the tile's first K steps last in its own.
+            constexpr bool kEarlyPartials = kHalf <= 32;
+            float pre[kEarlyPartials ? kHalf : 1];
+            const bool early = kEarlyPartials && w.kind == kOwner;
+            if constexpr (kEarlyPartials) {
+                if (early) {
+#pragma unroll
+                    for (int j = 0; j < kHalf; ++j) pre[j] = 0.0f;
+                    sum_partials<BN>(prm, w, blockIdx.x, 1, 0, etid, pre, abort);
+                }
+            }
             if (!mbar_wait(&acc_full[acc], acc_phase, &abort)) break;
             tc_fence_after();
             const int64_t prow = t.y_p + sub * 32 + lane;
@@ -606,6 +654,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (++acc == Cfg::kNumAcc) {
                 acc = 0;
                 acc_phase ^= 1u;
+            }
+            Work wf = w;
+            if constexpr (kEarlyPartials) {
+                if (early) {
+#pragma unroll
+                    for (int j = 0; j < kHalf; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + pre[j]);
+                    wf.kind = kFull;  // the partials are in: store like a whole tile
+                }
             }
             EpiCtx e;
             e.etid = etid;
@@ -622,7 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             e.p_end = t.p_end;
             e.q_end = t.q_end;
             e.staging = staging + (warp - 8) * 2048;
-            finish_item<BN, SWAP>(prm, &tmap_y, w, e, v, abort);
+            finish_item<BN, SWAP>(prm, &tmap_y, wf, e, v, abort);
         }
         if (lane == 0) bulk_wait_group<0>();  // output stores complete before the CTA exits
     }
