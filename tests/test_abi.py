@@ -124,3 +124,20 @@ def test_grouped_linear_validation_and_sizes():
     assert call(cp, 3, 256, wsb=1000) == -6
     z, zp = counts(0, 0, 0)
     assert call(zp, 3, 256, x=0, y=0, ws=0) == 0  # no token routed: nothing to do, nothing launched
+
+
+def test_noalloc_linear_validation():
+    """The no-allocation linear rejects bad arguments, and problems whose activation codes and
+    scales exceed its fixed scratch, before it touches the device."""
+    P = ctypes.c_void_p
+    lib = mq.load_library()
+    call = lambda M, K, N, x=FAKE, y=FAKE: lib.macaq_w4a4_linear_noalloc(P(x), M, K, P(FAKE), P(FAKE), P(FAKE), N,
+                                                                           P(y), None)
+    assert lib.macaq_w4a4_linear_noalloc(None, 4, 256, P(FAKE), P(FAKE), P(FAKE), 128, P(FAKE), None) == -1
+    assert call(0, 256, 128) == -2
+    assert call(4, 250, 128) == -2
+    assert call(4, 256, 0) == -2
+    assert call(4, 256, 128, x=MIS) == -3
+    assert call(4, 256, 128, y=MIS) == -3
+    # 65536 x 1024 activations: 32 MiB of codes alone, beyond the 32 MiB scratch
+    assert call(65536, 1024, 128) == -7
