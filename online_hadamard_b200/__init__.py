@@ -111,15 +111,27 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> None:
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, min_numel=None, device=None) -> None:
+    """Argument checks the C ABI cannot make (it sees bare pointers): a contiguous CUDA tensor of
+    the right dtype and shape or size, on the device of the call's other tensors.  A buffer
+    that is too small or on the wrong device would otherwise reach a kernel."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {device}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None:
+        _need_numel(t, name, min_numel)
+
+
+def _need_numel(t: torch.Tensor, name: str, n: int) -> None:
+    if t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call needs at least {n}")
 
 
 def scale_bytes(rows: int, K: int) -> int:
@@ -145,12 +157,12 @@ def macaq_calibrate_scale(xcal: torch.Tensor, W: torch.Tensor, s=None, stream=No
     """Per-channel scale s (fp32 [K]) from a bf16 calibration batch [C, K] and fp32 weights [N, K]."""
     C, K = xcal.shape
     _need(xcal, "xcal", torch.bfloat16)
-    _need(W, "W", torch.float32)
+    _need(W, "W", torch.float32, device=xcal.device)
     N = W.shape[0]
     if W.shape[1] != K:
         raise ValueError("xcal and W must have the same K")
     s = torch.empty(K, dtype=torch.float32, device=W.device) if s is None else s
-    _need(s, "s", torch.float32, (K,))
+    _need(s, "s", torch.float32, (K,), device=W.device)
     _check(load_library().macaq_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s), _stream(stream)),
            "macaq_calibrate_scale")
     return s
@@ -160,11 +172,14 @@ def macaq_fold_weights(W: torch.Tensor, s: torch.Tensor, Wq=None, Ws=None, act_m
     """Fold diag(s) H/sqrt(32) into W (fp32 [N, K]) and RTN-quantise: (Wq, Ws, act_mult)."""
     N, K = W.shape
     _need(W, "W", torch.float32)
-    _need(s, "s", torch.float32, (K,))
     dev = W.device
+    _need(s, "s", torch.float32, (K,), device=dev)
     Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=dev) if Wq is None else Wq
     Ws = torch.empty(max(scale_bytes(N, K), 1), dtype=torch.uint8, device=dev) if Ws is None else Ws
     act_mult = torch.empty(K, dtype=torch.float32, device=dev) if act_mult is None else act_mult
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
+    _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
     _check(load_library().macaq_fold_weights(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(Ws), _ptr(act_mult),
                                              _stream(stream)), "macaq_fold_weights")
     return Wq, Ws, act_mult
@@ -174,10 +189,12 @@ def macaq_act_transform_quant(x: torch.Tensor, act_mult: torch.Tensor, Aq=None, 
     """Scale, FWHT-32 and MXFP4-quantise bf16 activations [M, K]: (Aq, As)."""
     M, K = x.shape
     _need(x, "x", torch.bfloat16)
-    _need(act_mult, "act_mult", torch.float32, (K,))
     dev = x.device
+    _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
     Aq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Aq is None else Aq
     As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
+    _need(Aq, "Aq", torch.uint8, (M, K // 2), device=dev)
+    _need(As, "As", torch.uint8, min_numel=scale_bytes(M, K), device=dev)
     _check(load_library().macaq_act_transform_quant(_ptr(x), M, K, _ptr(act_mult), _ptr(Aq), _ptr(As),
                                                     _stream(stream)), "macaq_act_transform_quant")
     return Aq, As
@@ -190,6 +207,8 @@ def macaq_act_quant_plain(x: torch.Tensor, Aq=None, As=None, stream=None):
     dev = x.device
     Aq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev) if Aq is None else Aq
     As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
+    _need(Aq, "Aq", torch.uint8, (M, K // 2), device=dev)
+    _need(As, "As", torch.uint8, min_numel=scale_bytes(M, K), device=dev)
     _check(load_library().macaq_act_quant_plain(_ptr(x), M, K, _ptr(Aq), _ptr(As), _stream(stream)),
            "macaq_act_quant_plain")
     return Aq, As
@@ -201,18 +220,19 @@ def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: b
     workspace is allocated when not given (the schedule macaq_w4a4_linear uses);
     data_parallel=True passes none (data-parallel schedule)."""
     _need(Aq, "Aq", torch.uint8, (M, K // 2))
-    _need(Wq, "Wq", torch.uint8, (N, K // 2))
-    _need(As, "As", torch.uint8)
-    _need(Ws, "Ws", torch.uint8)
+    dev = Aq.device
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(As, "As", torch.uint8, min_numel=scale_bytes(M, K), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
     dt = torch.float32 if out_fp32 else torch.bfloat16
-    y = torch.empty(M, N, dtype=dt, device=Aq.device) if y is None else y
-    _need(y, "y", dt, (M, N))
+    y = torch.empty(M, N, dtype=dt, device=dev) if y is None else y
+    _need(y, "y", dt, (M, N), device=dev)
     if data_parallel:
         workspace = None
     elif workspace is None:
-        workspace = torch.empty(max(gemm_workspace_bytes(M, N, K), 1), dtype=torch.uint8, device=Aq.device)
+        workspace = torch.empty(max(gemm_workspace_bytes(M, N, K), 1), dtype=torch.uint8, device=dev)
     if workspace is not None:
-        _need(workspace, "workspace", torch.uint8)
+        _need(workspace, "workspace", torch.uint8, device=dev)
     _check(load_library().macaq_mxfp4_gemm(_ptr(Aq), _ptr(As), M, _ptr(Wq), _ptr(Ws), N, K, _ptr(y),
                                            1 if out_fp32 else 0, _ptr(workspace),
                                            0 if workspace is None else workspace.numel(), _stream(stream)),
@@ -225,14 +245,15 @@ def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor,
     """y = x W^T through the online transform, MXFP4 quantisation and the W4A4 GEMM (bf16 [M, N])."""
     M, K = x.shape
     _need(x, "x", torch.bfloat16)
-    _need(act_mult, "act_mult", torch.float32, (K,))
-    _need(Wq, "Wq", torch.uint8, (N, K // 2))
-    _need(Ws, "Ws", torch.uint8)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
-    _need(y, "y", torch.bfloat16, (M, N))
+    dev = x.device
+    _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N), device=dev)
     need = linear_workspace_bytes(M, N, K)
-    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
-    _need(workspace, "workspace", torch.uint8)
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, device=dev)
     _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
                                             _ptr(workspace), workspace.numel(), _stream(stream)),
            "macaq_w4a4_linear")
@@ -244,13 +265,14 @@ def macaq_mxfp4_linear(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: i
     """Plain MXFP4 linear (no scale, no transform): the baseline of the transform's overhead."""
     M, K = x.shape
     _need(x, "x", torch.bfloat16)
-    _need(Wq, "Wq", torch.uint8, (N, K // 2))
-    _need(Ws, "Ws", torch.uint8)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
-    _need(y, "y", torch.bfloat16, (M, N))
+    dev = x.device
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N), device=dev)
     need = linear_workspace_bytes(M, N, K)
-    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
-    _need(workspace, "workspace", torch.uint8)
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, device=dev)
     _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
                                              workspace.numel(), _stream(stream)), "macaq_mxfp4_linear")
     return y
@@ -279,15 +301,16 @@ def macaq_w4a4_grouped_linear(x: torch.Tensor, counts, act_mult, Wq: torch.Tenso
     if int(c.sum()) != T:
         raise ValueError("counts must sum to the rows of x")
     _need(x, "x", torch.bfloat16)
+    dev = x.device
     if act_mult is not None:
-        _need(act_mult, "act_mult", torch.float32, (E, K))
-    _need(Wq, "Wq", torch.uint8, (E, N, K // 2))
-    _need(Ws, "Ws", torch.uint8)
-    y = torch.empty(T, N, dtype=torch.bfloat16, device=x.device) if y is None else y
-    _need(y, "y", torch.bfloat16, (T, N))
+        _need(act_mult, "act_mult", torch.float32, (E, K), device=dev)
+    _need(Wq, "Wq", torch.uint8, (E, N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=E * scale_bytes(N, K), device=dev)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (T, N), device=dev)
     need = max(grouped_workspace_bytes(c, N, K), 1)
-    workspace = torch.empty(need, dtype=torch.uint8, device=x.device) if workspace is None else workspace
-    _need(workspace, "workspace", torch.uint8)
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, device=dev)
     _check(load_library().macaq_w4a4_grouped_linear(_ptr(x), cp, E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N,
                                                     _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
            "macaq_w4a4_grouped_linear")
@@ -305,11 +328,12 @@ def macaq_w4a4_linear_noalloc(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch
     only when the caller does not pass it."""
     M, K = x.shape
     _need(x, "x", torch.bfloat16)
-    _need(act_mult, "act_mult", torch.float32, (K,))
-    _need(Wq, "Wq", torch.uint8, (N, K // 2))
-    _need(Ws, "Ws", torch.uint8)
-    y = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if y is None else y
-    _need(y, "y", torch.bfloat16, (M, N))
+    dev = x.device
+    _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, N), device=dev)
     _check(load_library().macaq_w4a4_linear_noalloc(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
                                                     _stream(stream)), "macaq_w4a4_linear_noalloc")
     return y

@@ -141,3 +141,20 @@ def test_noalloc_linear_validation():
     assert call(4, 256, 128, y=MIS) == -3
     # 65536 x 1024 activations: 32 MiB of codes alone, beyond the 32 MiB scratch
     assert call(65536, 1024, 128) == -7
+
+
+def test_binding_refuses_host_tensors_and_short_buffers():
+    """The Python binding hands the library bare pointers, so it checks what the C ABI cannot:
+    host tensors are refused (there is no CPU path), and a buffer shorter than the call needs
+    is refused before any pointer reaches a kernel."""
+    import pytest
+    import torch
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mq.macaq_act_transform_quant(x, torch.ones(256))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mq.macaq_w4a4_linear(x, torch.ones(256), torch.zeros(128, 128, dtype=torch.uint8),
+                             torch.zeros(mq.scale_bytes(128, 256), dtype=torch.uint8), 128)
+    with pytest.raises(ValueError, match="needs at least"):
+        mq._need_numel(torch.zeros(mq.scale_bytes(128, 256) - 1, dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
+    mq._need_numel(torch.zeros(mq.scale_bytes(128, 256), dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
