@@ -2,7 +2,8 @@
 
 Argument marshalling only: every function below checks tensor placement, dtype and
 contiguity, allocates outputs with torch when the caller does not pass them, and calls the
-C entry point of the same name in ``_build/libmacaq.so`` on the current CUDA stream.  All
+C entry point of the same name in ``_build/libmacaq.so`` with the tensors' device made
+current, on that device's current CUDA stream (or the stream passed, which must belong to it).  All
 arithmetic runs in the library's CUDA kernels; there is no CPU or PyTorch fallback -- if
 the library cannot be loaded, every call raises.
 
@@ -13,6 +14,7 @@ conventions are documented in include/macaq.h.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -105,10 +107,26 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device: torch.device) -> ctypes.c_void_p:
+    """The CUDA stream handle of a call whose tensors live on `device`: the given stream, which
+    must belong to that device, or that device's current stream."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    else:
+        _check_stream_device(stream, device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_stream_device(stream, device: torch.device) -> None:
+    """A stream of another GPU would run the kernels there, on pointers into this one."""
+    sdev = torch.device(stream.device)
+    if sdev.type != "cuda" or sdev.index != device.index:
+        raise ValueError(f"stream belongs to {sdev}, the call's tensors to {device}")
+
+
+def _device(device):
+    """`device` made current for the library call inside (None: the current device as it is)."""
+    return contextlib.nullcontext() if device is None else torch.cuda.device(device)
 
 
 def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, min_numel=None, device=None) -> None:
@@ -143,28 +161,33 @@ def scale_offset(r: int, kb: int, K: int) -> int:
     return int(load_library().macaq_scale_offset(r, kb, K))
 
 
-def linear_workspace_bytes(M: int, N: int, K: int) -> int:
-    """Scratch bytes macaq_w4a4_linear and macaq_mxfp4_linear need on the current device."""
-    return int(load_library().macaq_linear_workspace_bytes(M, N, K))
+def linear_workspace_bytes(M: int, N: int, K: int, device=None) -> int:
+    """Scratch bytes macaq_w4a4_linear and macaq_mxfp4_linear need on `device` (default: the
+    current CUDA device; the size depends on its SM count)."""
+    with _device(device):
+        return int(load_library().macaq_linear_workspace_bytes(M, N, K))
 
 
-def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
-    """Scratch bytes of the GEMM's stream-K schedule on the current device."""
-    return int(load_library().macaq_gemm_workspace_bytes(M, N, K))
+def gemm_workspace_bytes(M: int, N: int, K: int, device=None) -> int:
+    """Scratch bytes of the GEMM's stream-K schedule on `device` (default: the current one)."""
+    with _device(device):
+        return int(load_library().macaq_gemm_workspace_bytes(M, N, K))
 
 
 def macaq_calibrate_scale(xcal: torch.Tensor, W: torch.Tensor, s=None, stream=None):
     """Per-channel scale s (fp32 [K]) from a bf16 calibration batch [C, K] and fp32 weights [N, K]."""
     C, K = xcal.shape
     _need(xcal, "xcal", torch.bfloat16)
-    _need(W, "W", torch.float32, device=xcal.device)
+    dev = xcal.device
+    _need(W, "W", torch.float32, device=dev)
     N = W.shape[0]
     if W.shape[1] != K:
         raise ValueError("xcal and W must have the same K")
     s = torch.empty(K, dtype=torch.float32, device=W.device) if s is None else s
     _need(s, "s", torch.float32, (K,), device=W.device)
-    _check(load_library().macaq_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s), _stream(stream)),
-           "macaq_calibrate_scale")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s), _stream(stream, dev)),
+               "macaq_calibrate_scale")
     return s
 
 
@@ -180,8 +203,9 @@ def macaq_fold_weights(W: torch.Tensor, s: torch.Tensor, Wq=None, Ws=None, act_m
     _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
     _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
     _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
-    _check(load_library().macaq_fold_weights(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(Ws), _ptr(act_mult),
-                                             _stream(stream)), "macaq_fold_weights")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_fold_weights(_ptr(W), N, K, _ptr(s), _ptr(Wq), _ptr(Ws), _ptr(act_mult),
+                                                 _stream(stream, dev)), "macaq_fold_weights")
     return Wq, Ws, act_mult
 
 
@@ -195,8 +219,9 @@ def macaq_act_transform_quant(x: torch.Tensor, act_mult: torch.Tensor, Aq=None, 
     As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
     _need(Aq, "Aq", torch.uint8, (M, K // 2), device=dev)
     _need(As, "As", torch.uint8, min_numel=scale_bytes(M, K), device=dev)
-    _check(load_library().macaq_act_transform_quant(_ptr(x), M, K, _ptr(act_mult), _ptr(Aq), _ptr(As),
-                                                    _stream(stream)), "macaq_act_transform_quant")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_act_transform_quant(_ptr(x), M, K, _ptr(act_mult), _ptr(Aq), _ptr(As),
+                                                        _stream(stream, dev)), "macaq_act_transform_quant")
     return Aq, As
 
 
@@ -209,8 +234,9 @@ def macaq_act_quant_plain(x: torch.Tensor, Aq=None, As=None, stream=None):
     As = torch.empty(max(scale_bytes(M, K), 1), dtype=torch.uint8, device=dev) if As is None else As
     _need(Aq, "Aq", torch.uint8, (M, K // 2), device=dev)
     _need(As, "As", torch.uint8, min_numel=scale_bytes(M, K), device=dev)
-    _check(load_library().macaq_act_quant_plain(_ptr(x), M, K, _ptr(Aq), _ptr(As), _stream(stream)),
-           "macaq_act_quant_plain")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_act_quant_plain(_ptr(x), M, K, _ptr(Aq), _ptr(As), _stream(stream, dev)),
+               "macaq_act_quant_plain")
     return Aq, As
 
 
@@ -230,13 +256,14 @@ def macaq_mxfp4_gemm(Aq, As, Wq, Ws, M: int, N: int, K: int, y=None, out_fp32: b
     if data_parallel:
         workspace = None
     elif workspace is None:
-        workspace = torch.empty(max(gemm_workspace_bytes(M, N, K), 1), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(max(gemm_workspace_bytes(M, N, K, dev), 1), dtype=torch.uint8, device=dev)
     if workspace is not None:
         _need(workspace, "workspace", torch.uint8, device=dev)
-    _check(load_library().macaq_mxfp4_gemm(_ptr(Aq), _ptr(As), M, _ptr(Wq), _ptr(Ws), N, K, _ptr(y),
-                                           1 if out_fp32 else 0, _ptr(workspace),
-                                           0 if workspace is None else workspace.numel(), _stream(stream)),
-           "macaq_mxfp4_gemm")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_mxfp4_gemm(_ptr(Aq), _ptr(As), M, _ptr(Wq), _ptr(Ws), N, K, _ptr(y),
+                                               1 if out_fp32 else 0, _ptr(workspace),
+                                               0 if workspace is None else workspace.numel(), _stream(stream, dev)),
+               "macaq_mxfp4_gemm")
     return y
 
 
@@ -251,12 +278,13 @@ def macaq_w4a4_linear(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch.Tensor,
     _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
     _need(y, "y", torch.bfloat16, (M, N), device=dev)
-    need = linear_workspace_bytes(M, N, K)
+    need = linear_workspace_bytes(M, N, K, dev)
     workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _need(workspace, "workspace", torch.uint8, device=dev)
-    _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
-                                            _ptr(workspace), workspace.numel(), _stream(stream)),
-           "macaq_w4a4_linear")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_w4a4_linear(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+                                                _ptr(workspace), workspace.numel(), _stream(stream, dev)),
+               "macaq_w4a4_linear")
     return y
 
 
@@ -270,11 +298,12 @@ def macaq_mxfp4_linear(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: i
     _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
     _need(y, "y", torch.bfloat16, (M, N), device=dev)
-    need = linear_workspace_bytes(M, N, K)
+    need = linear_workspace_bytes(M, N, K, dev)
     workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _need(workspace, "workspace", torch.uint8, device=dev)
-    _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
-                                             workspace.numel(), _stream(stream)), "macaq_mxfp4_linear")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
+                                                 workspace.numel(), _stream(stream, dev)), "macaq_mxfp4_linear")
     return y
 
 
@@ -311,9 +340,10 @@ def macaq_w4a4_grouped_linear(x: torch.Tensor, counts, act_mult, Wq: torch.Tenso
     need = max(grouped_workspace_bytes(c, N, K), 1)
     workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
     _need(workspace, "workspace", torch.uint8, device=dev)
-    _check(load_library().macaq_w4a4_grouped_linear(_ptr(x), cp, E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N,
-                                                    _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)),
-           "macaq_w4a4_grouped_linear")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_w4a4_grouped_linear(_ptr(x), cp, E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N,
+                                                        _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream, dev)),
+               "macaq_w4a4_grouped_linear")
     return y
 
 
@@ -334,8 +364,9 @@ def macaq_w4a4_linear_noalloc(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch
     _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if y is None else y
     _need(y, "y", torch.bfloat16, (M, N), device=dev)
-    _check(load_library().macaq_w4a4_linear_noalloc(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
-                                                    _stream(stream)), "macaq_w4a4_linear_noalloc")
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_w4a4_linear_noalloc(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+                                                        _stream(stream, dev)), "macaq_w4a4_linear_noalloc")
     return y
 
 

@@ -20,8 +20,16 @@
 //   * every call shares it and it keeps the previous call's contents.  Nothing in it has
 //     to start at zero: each call writes every code byte and every scale byte of its real
 //     rows before reading them, a stream-K flag counts only when it holds the tag of the
-//     current launch (and each launch clears the flags it consumed), and the bytes it does not write (padded rows of the last 128-row scale atom, stale
-//     partial sums) are never used for a stored output;
+//     current launch (and each launch clears the flags it consumed), and the bytes it does
+//     not write (padded rows of the last 128-row scale atom, stale partial sums) are never
+//     used for a stored output;
+//   * the stream-K flag words sit after each call's own activation bytes, so their offset
+//     changes with the shape, and a later call of another shape may find an earlier call's
+//     flag words among its activation codes or its own flags at bytes an earlier call used
+//     for codes.  None of that needs clearing: the library never reuses a launch tag (a
+//     per-process random start, one step per launch), except when a CUDA graph replays a
+//     captured launch of the same call, whose flags sit at the same place and were cleared
+//     by the launch that consumed them;
 //   * two calls whose kernels overlap on the GPU (different streams without ordering, or
 //     several host threads) race on the array and corrupt each other's results: order
 //     them on one stream or serialise them;

@@ -240,7 +240,6 @@ void oracle_mx_gemm(const uint8_t* Aq, const uint8_t* As, const int64_t* rows, i
     free(a);
 }
 
-/* Number of OpenMP threads the oracle runs with (reported beside its timings). */
 /* Per-channel scale from a calibration batch xcal [C][K] (bf16 values held in fp32) and the
  * weights W [N][K]: column maxima of |.|, then sqrt of their quotient in double, rounded once to
  * fp32; 1 for a column whose activation or weight maximum is zero. */
@@ -253,6 +252,7 @@ void oracle_calibrate_scale(const float* xcal, int64_t C, const float* W, int64_
     }
 }
 
+/* Number of OpenMP threads the oracle runs with (reported beside its timings). */
 int oracle_num_threads(void) {
     int n = 1;
 #pragma omp parallel

@@ -158,3 +158,20 @@ def test_binding_refuses_host_tensors_and_short_buffers():
     with pytest.raises(ValueError, match="needs at least"):
         mq._need_numel(torch.zeros(mq.scale_bytes(128, 256) - 1, dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
     mq._need_numel(torch.zeros(mq.scale_bytes(128, 256), dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
+
+
+def test_binding_refuses_a_stream_of_another_device():
+    """Kernels run on the stream's device: a stream of another GPU than the tensors' would make
+    them read this GPU's memory through pointers the other one cannot use, so it is refused
+    before the call."""
+    import types
+
+    import pytest
+    import torch
+    dev0 = torch.device("cuda", 0)
+    with pytest.raises(ValueError, match="stream belongs to cuda:1"):
+        mq._check_stream_device(types.SimpleNamespace(device=torch.device("cuda", 1)), dev0)
+    with pytest.raises(ValueError, match="stream belongs to cpu"):
+        mq._check_stream_device(types.SimpleNamespace(device=torch.device("cpu")), dev0)
+    mq._check_stream_device(types.SimpleNamespace(device=torch.device("cuda", 0)), dev0)
+    mq._check_stream_device(types.SimpleNamespace(device="cuda:0"), dev0)
