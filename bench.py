@@ -4,17 +4,19 @@
 
 One step = one forward pass of the layer's hot path over one batch: the online per-channel
 scale + FWHT-32 + MXFP4 quantisation of the bf16 activations feeding the block-scaled
-MXFP4 GEMM (macaq_w4a4_linear), on the Llama-3-8B-shaped MLP up projection at prefill
-(M=2048, K=4096, N=14336) with seeded synthetic inputs (workloads.py).  The weight fold is
-offline and timed separately.  Inputs rotate over enough copies that the bytes touched
-between two uses of a copy exceed the 126 MB L2, so every step streams from HBM.
+MXFP4 GEMM (macaq_w4a4_linear), on the Qwen3-32B-shaped MLP down projection at prefill
+(M=4096, K=25600, N=5120; the largest single-GPU workload) with seeded synthetic inputs
+(workloads.py).  The weight fold is offline and timed separately.  Inputs rotate over copies
+whose bytes each exceed the 126 MB L2, so every step streams from HBM.
 
 Printed on rank 0: one JSON line with the whole-job TFLOP/s, the roofline of the dominant
 kernel (the tcgen05 GEMM, timed live with CUDA events), the online-transform overhead over
 plain MXFP4 (macaq_mxfp4_linear: plain quantisation + the same GEMM) and over the GEMM alone, an end-to-end
 figure through the C ABI with host buffers, the oracle's CPU throughput on a bounded
-sample, SM clocks sampled during the timed region, and secondary workloads (decode and
-the Qwen3-32B-shaped down projection).
+sample (whose rows are also compared with the GPU's codes, scales and outputs), SM clocks
+sampled during the timed region, the secondary workloads (the Llama-3-8B up projection,
+decode, the 64-layer stack, grouped MoE linears) and, last, a compact summary of every
+workload's figures.
 
 --impl reference times the CPU oracle (the reference arm of this repository) on a bounded
 sample of the same workload.  With N > 1 GPUs (torchrun), each rank runs an independent
@@ -116,8 +118,11 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
+        d["_source"] = "measured"
         return d, "measured"
-    return dict(PEAKS_FALLBACK), "fallback"
+    d = dict(PEAKS_FALLBACK)
+    d["_source"] = "fallback"
+    return d, "fallback"
 
 
 def file_hash(path):
@@ -331,34 +336,97 @@ def time_ab(fns, steps, warmup, device, rounds=5):
 # --------------------------------------------------------------------------- CPU baseline
 
 
-def cpu_baseline(wl, min_seconds=10.0, max_passes=8):
-    """The oracle as it stands, on the host cores: transform + quantise every activation row
-    and contract them with the folded weights (the fold is offline and excluded), repeated
-    over whole passes of the workload until at least `min_seconds` of CPU work."""
+def _scale_index(rows, K):
+    """Offsets of (row, 32-block) in the library's E8M0 "MMA tile layout" (include/macaq.h)."""
+    kbp = 8 * ((K + 255) // 256)
+    r = np.asarray(rows, dtype=np.int64)[:, None]
+    kb = np.arange(K // 32, dtype=np.int64)[None, :]
+    return ((r // 128) * (kbp // 4) + kb // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + kb % 4
+
+
+def _mx_diff(codes, scales, ref_codes, ref_scales, V):
+    """Mismatching MXFP4 codes and E8M0 scales of the GPU against the oracle, and how many of
+    them are exempt: the oracle's fp32 value within 1 ulp of a rounding boundary of the E2M1
+    grid (or the block maximum within 1 ulp of a power of two, for a scale).  V (the oracle's
+    fp32 values before rounding, or a callable giving them) is used only when something differs."""
+    g = np.stack([codes & 0xF, codes >> 4], -1).reshape(codes.shape[0], -1)
+    r = np.stack([ref_codes & 0xF, ref_codes >> 4], -1).reshape(codes.shape[0], -1)
+    bad_c, bad_s = g != r, scales != ref_scales
+    out = {"codes": int(g.size), "code_mismatch": int(bad_c.sum()), "scales": int(bad_s.size),
+           "scale_mismatch": int(bad_s.sum()), "exempt": 0}
+    if bad_c.any() or bad_s.any():
+        a = np.abs((V() if callable(V) else V).astype(np.float32))
+        lo = np.nextafter(a, np.float32(0)).astype(np.float64)
+        hi = np.nextafter(a, np.float32(np.inf)).astype(np.float64)
+        sc = np.exp2(np.repeat(ref_scales, 32, axis=1).astype(np.float64) - 127)
+        near = np.zeros(a.shape, bool)
+        for t in (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0):
+            near |= (lo <= t * sc) & (t * sc <= hi)
+        amax = a.reshape(a.shape[0], -1, 32).max(-1)
+        ex = lambda v: (v.view(np.uint32) >> 23) & 0xFF
+        near_s = (ex(np.nextafter(amax, np.float32(np.inf))) != ex(amax)) | \
+                 (ex(np.nextafter(amax, np.float32(0))) != ex(amax))
+        out["exempt"] = int((bad_c & near).sum() + (bad_s & near_s).sum())
+    return out
+
+
+def cpu_baseline(wl, gpu, min_seconds=10.0, rows_per_pass=128, max_passes=64):
+    """The oracle as it stands, on the host cores: transform + quantise a seeded sample of
+    activation rows and contract them with the folded weights (fp64), one new sample of
+    `rows_per_pass` rows per pass, until at least `min_seconds` of CPU work (the fold is
+    offline and excluded).  The first sample's codes, scales and outputs are compared with the
+    GPU's for the same rows (`gpu`: device tensors of the timed layer), and the GPU's weight
+    fold with the oracle's: bit-exact codes and scales (near-boundary mismatches counted as
+    exempt), y within a relative Frobenius error of 1e-3 of the bf16-rounded exact result."""
     import oracle
     W = wls.make_w(wl)
     s = wls.make_s(wl, W)
     x = wls.make_x(wl)
-    Wq, Ws, a = oracle.fold_weights(W.numpy(), s.numpy())
+    Wf = W.numpy()
+    del W
+    Wq, Ws, a = oracle.fold_weights(Wf, s.numpy())
     xs = x.float().numpy()
-    passes, dt = 0, 0.0
-    while passes < max_passes and (passes == 0 or dt < min_seconds):
+    rpp = min(rows_per_pass, wl.M)
+    perm = np.random.default_rng(4).permutation(wl.M)
+    passes, dt, first = 0, 0.0, None
+    while passes < max_passes and (passes == 0 or dt < min_seconds) and (passes + 1) * rpp <= wl.M:
+        idx = np.sort(perm[passes * rpp:(passes + 1) * rpp])
         t0 = time.perf_counter()
-        Aq, As = oracle.act_transform_quant(xs, a)
-        oracle.mx_gemm(Aq, As, Wq, Ws)
+        Aq, As = oracle.act_transform_quant(xs[idx], a)
+        y = oracle.mx_gemm(Aq, As, Wq, Ws)
         dt += time.perf_counter() - t0
+        if first is None:
+            first = (idx, Aq, As, y)
         passes += 1
-    flops = passes * wl.flops
+    flops = passes * 2.0 * rpp * wl.N * wl.K
+    idx, Aq, As, y = first
+    V = oracle.transform_f32(xs[idx], a)
+    g_codes = gpu["Aq"][torch.as_tensor(idx, device=gpu["Aq"].device)].cpu().numpy()
+    g_scales = gpu["As"].cpu().numpy()[_scale_index(idx, wl.K)]
+    act = _mx_diff(g_codes, g_scales, Aq, As, V)
+    w_scales = gpu["Ws"].cpu().numpy()[_scale_index(np.arange(wl.N), wl.K)]
+    w = _mx_diff(gpu["Wq"].cpu().numpy(), w_scales, Wq, Ws,
+                 lambda: oracle.transform_f32(Wf, oracle.multipliers(s.numpy())[1]))
+    gy = gpu["y"][torch.as_tensor(idx, device=gpu["y"].device)].double().cpu().numpy()
+    ref = torch.from_numpy(y).to(torch.float32).to(torch.bfloat16).double().numpy()
+    rel = float(np.linalg.norm(gy - ref) / np.linalg.norm(ref))
+    parity = {"rows": int(len(idx)), "activations": act, "weights": w, "y_rel_fro_vs_oracle": rel,
+              "y_tolerance": 1e-3, "ok": bool(rel <= 1e-3 and all(d["code_mismatch"] + d["scale_mismatch"] == d["exempt"]
+                                                                  for d in (act, w)))}
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{passes} full pass(es) of {wl.name} ({wl.M} rows: transform+quant+fp64 GEMM), {dt:.1f} s",
-            "seconds": dt}
+            "sample": f"{passes} sample(s) of {rpp} of the {wl.M} rows of {wl.name} "
+                      f"(transform+quant+fp64 GEMM against all {wl.N} outputs), {dt:.1f} s",
+            "seconds": dt, "parity": parity}
+
+
+HEADLINE = wls.QWEN_DOWN  # the largest single-GPU workload
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = wls.LLAMA_UP
+    wl = HEADLINE
     import oracle
     W = wls.make_w(wl)
     s = wls.make_s(wl, W)
@@ -422,7 +490,7 @@ def main():
     peaks, peak_src = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
 
-    wl = wls.LLAMA_UP
+    wl = HEADLINE
     layer = Layer(mq, wl, device)
 
     barrier = ranks.barrier
@@ -446,7 +514,7 @@ def main():
     while time.perf_counter() - t_soak < 0.4:
         loop.graph.replay()
         soak += 1
-        if soak % 8 == 0:
+        if soak % 4 == 0:
             torch.cuda.synchronize(device)
     torch.cuda.synchronize(device)
     clk = clocks.stop()
@@ -457,14 +525,9 @@ def main():
 
     # ---- dominant kernel, the comparators and end to end (same rotation); the overhead
     # compares medians of alternating replays of the W4A4 and plain-MXFP4 linears
-    ab = time_ab({"linear": layer.linear, "plain": layer.plain, "gemm": layer.gemm,
-                  "transform": layer.transform_only}, args.steps, args.warmup, device)
-    ms_gemm, ms_plain, ms_xform, ms_lin_ab = ab["gemm"], ab["plain"], ab["transform"], ab["linear"]
+    head = prefill_leg(layer, args, peaks)
     e2e_steps = max(3, min(args.steps, 10))
     ms_e2e = max_over_ranks(time_eager(layer.e2e, e2e_steps, 3, device))
-    gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
-    xform_bytes = wl.M * wl.K * 2 + wl.M * wl.K * (0.5 + 1 / 32) + wl.K * 4
-    traffic = recorded_traffic("mxf4_gemm_pair_256x256:" + wl.name)
 
     extra = {}
     if not args.no_extra:
@@ -475,7 +538,10 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(wl)
+        layer.linear(0)
+        torch.cuda.synchronize(device)
+        cpu = cpu_baseline(wl, {"Aq": layer.Aq[0], "As": layer.As[0], "Wq": layer.Wq[0], "Ws": layer.Ws[0],
+                                "y": layer.y[0]})
 
     if rank == 0:
         out = {
@@ -483,28 +549,83 @@ def main():
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "mxfp4 (e2m1 x e2m1, ue8m0 scales, fp32 accumulate, bf16 out)", "data": "synthetic",
-            "config": headline_config(wl, world, f"inputs rotated over {layer.copies} copies (> 3x L2)"),
-            "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<5> (2-CTA 256x256 tiles, scale warps)", "achieved": gemm_tflops,
-                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} (fp4:bf16 nominal)",
-                         "ms_per_launch": ms_gemm},
+            "config": headline_config(wl, world, f"inputs rotated over {layer.copies} copies, each > L2"),
+            "roofline": head["roofline"],
             "linear_roofline": linear_roofline(wl, ms, fp4_peak, peaks["hbm_gbs"]),
-            "overhead": {"linear_ms": ms_lin_ab, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
-                         "vs_plain_mxfp4_pct": 100.0 * (ms_lin_ab / ms_plain - 1.0),
-                         "vs_gemm_only_pct": 100.0 * (ms_lin_ab / ms_gemm - 1.0),
-                         "method": "medians of 5 alternating graph replays per variant",
-                         "transform_quant_ms": ms_xform,
-                         "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
+            "overhead": head["overhead"],
             "e2e": {"value": whole_job_tflops(world, wl.flops, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                     "h2d_bytes_per_step": wl.M * wl.K * 2, "d2h_bytes_per_step": wl.M * wl.N * 2},
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
             "fold_ms": layer.fold_s * 1e3,
             "cpu_baseline": cpu,
+            "parity": cpu["parity"] if cpu else None,
             "secondary": extra,
         }
+        out["summary"] = summary(out)
         print(json.dumps(out))
     ranks.close()
+
+
+def prefill_leg(layer, args, peaks):
+    """A prefill linear's dominant kernel (the 2-CTA GEMM, timed alone on the same rotation) and
+    the transform's overhead against plain MXFP4 and the GEMM alone, from medians of alternating
+    graph replays of the four variants."""
+    wl, device = layer.wl, layer.dev
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    ab = time_ab({"linear": layer.linear, "plain": layer.plain, "gemm": layer.gemm,
+                  "transform": layer.transform_only}, args.steps, args.warmup, device)
+    ms_gemm, ms_plain, ms_xform, ms_lin = ab["gemm"], ab["plain"], ab["transform"], ab["linear"]
+    gemm_tflops = wl.flops / (ms_gemm * 1e-3) / 1e12
+    xform_bytes = wl.M * wl.K * 2 + wl.M * wl.K * (0.5 + 1 / 32) + wl.K * 4
+    peak_src = peaks.get("_source", "measured")
+    return {
+        "roofline": {"bound": "tensor", "kernel": "mxf4_gemm_pair_kernel<5> (2-CTA 256x256 tiles, scale warps)",
+                     "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
+                     "traffic": recorded_traffic("mxf4_gemm_pair_256x256:" + wl.name),
+                     "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} x {FP4_OVER_BF16} "
+                                    "(fp4:bf16 nominal)",
+                     "ms_per_launch": ms_gemm},
+        "overhead": {"linear_ms": ms_lin, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
+                     "vs_plain_mxfp4_pct": 100.0 * (ms_lin / ms_plain - 1.0),
+                     "vs_gemm_only_pct": 100.0 * (ms_lin / ms_gemm - 1.0),
+                     "method": "medians of 5 alternating graph replays per variant",
+                     "transform_quant_ms": ms_xform,
+                     "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
+    }
+
+
+def summary(out):
+    """Every workload's key figures, rounded, in a few hundred characters (the end of the line)."""
+    r = lambda v, n=3: None if v is None else float(f"{v:.{n}g}")
+    sm = {"cfg4_down_prefill": {"tflops": r(out["value"]), "linear_roof": r(out["linear_roofline"]["frac"]),
+                                "gemm_roof": r(out["roofline"]["frac"]),
+                                "ovh_plain_pct": r(out["overhead"]["vs_plain_mxfp4_pct"], 2),
+                                "ovh_gemm_pct": r(out["overhead"]["vs_gemm_only_pct"], 2)}}
+    sec = out.get("secondary") or {}
+    for k, v in sec.items():
+        if k.startswith("llama3_8b_up_prefill"):
+            sm["cfg2_llama_up"] = {"tflops": r(v["tflops"]), "linear_roof": r(v["linear_roofline"]["frac"]),
+                                   "gemm_roof": r(v["roofline"]["frac"]),
+                                   "ovh_plain_pct": r(v["overhead"]["vs_plain_mxfp4_pct"], 2),
+                                   "ovh_gemm_pct": r(v["overhead"]["vs_gemm_only_pct"], 2)}
+        elif k.startswith("qwen3_32b_up_decode"):
+            sm["cfg3_" + k.split("_")[-1]] = {"gbs": r(v["gbs"]), "linear_roof": r(v["linear_roofline"]["frac"]),
+                                              "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2)}
+    st = sec.get("qwen3_32b_stack") or {}
+    for k, v in st.items():
+        if k.startswith("M"):
+            sm["cfg5_" + k] = {"ms": r(v["w4a4_ms"]), "roof": r(v["linear_roofline_frac"]),
+                               "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2)}
+    for k, v in (sec.get("qwen3_moe_grouped") or {}).items():
+        if isinstance(v, dict):
+            sm["moe_" + k] = {"us": r(v["ms"] * 1e3), "roof": r(v["linear_roofline_frac"]),
+                              "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2)}
+    par = out.get("parity")
+    if par:
+        sm["parity_cfg4"] = {"ok": par["ok"], "exempt": par["activations"]["exempt"] + par["weights"]["exempt"],
+                             "y_rel": r(par["y_rel_fro_vs_oracle"], 2)}
+    return sm
 
 
 def profile_kernels(name):
@@ -625,8 +746,17 @@ def moe_sweep(mq, device, peaks, token_counts=(16, 4096), steps=10, warmup=3):
 
 
 def secondary(mq, device, peaks, args):
-    """Decode (HBM-bound) and the Qwen3-32B down projection (tensor-bound)."""
+    """The Llama-3-8B up projection (tensor-bound prefill) and decode (HBM-bound)."""
     res = {}
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    wl = wls.LLAMA_UP
+    layer = Layer(mq, wl, device)
+    leg = prefill_leg(layer, args, peaks)
+    ms = leg["overhead"]["linear_ms"]
+    res[wl.name] = {"ms": ms, "tflops": wl.flops / (ms * 1e-3) / 1e12,
+                    "linear_roofline": linear_roofline(wl, ms, fp4_peak, peaks["hbm_gbs"]), **leg}
+    del layer
+    torch.cuda.empty_cache()
     steps = max(10, args.steps // 2)
     for M in wls.QWEN_DECODE_M:
         wl = wls.QWEN_UP_DECODE.with_m(M)
@@ -640,16 +770,6 @@ def secondary(mq, device, peaks, args):
                                    "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
         del layer
         torch.cuda.empty_cache()
-    wl = wls.QWEN_DOWN
-    layer = Layer(mq, wl, device, copies=2)
-    ab = time_ab({"linear": layer.linear, "plain": layer.plain, "gemm": layer.gemm}, steps, args.warmup, device)
-    ms, ms_plain, ms_gemm = ab["linear"], ab["plain"], ab["gemm"]
-    t = wl.flops / (ms * 1e-3) / 1e12
-    res[wl.name] = {"ms": ms, "tflops": t, "frac_fp4_peak": t / (peaks["bf16_tflops"] * FP4_OVER_BF16),
-                    "linear_roofline": linear_roofline(wl, ms, peaks["bf16_tflops"] * FP4_OVER_BF16, peaks["hbm_gbs"]),
-                    "gemm_ms": ms_gemm, "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0)}
-    del layer
-    torch.cuda.empty_cache()
     return res
 
 

@@ -42,10 +42,32 @@ def _near_code_boundary(v: np.ndarray, e: np.ndarray) -> np.ndarray:
     return res
 
 
-def compare_mx(gpu_codes, gpu_scales_tiled, ref_codes, ref_scales, rows, K, V=None):
+# Comparisons of codes and scales made in this test session, per label (the config they cover):
+# printed at the end of the run by the terminal-summary hook in tests/conftest.py, so the
+# counts of exempt near-boundary mismatches appear in the run's log.
+PARITY_LOG: dict = {}
+
+
+def config_label(wl, what: str) -> str:
+    """Label of a comparison: the workload's config number and what was compared."""
+    return f"config {wl.config} {what}"
+
+
+def _record(label, stats):
+    if label is None:
+        return
+    tot = PARITY_LOG.setdefault(label, {"codes": 0, "scales": 0, "code_mismatch": 0, "scale_mismatch": 0,
+                                        "exempt": 0})
+    for k in tot:
+        tot[k] += stats[k]
+
+
+def compare_mx(gpu_codes, gpu_scales_tiled, ref_codes, ref_scales, rows, K, V=None, label=None):
     """Bit-exact comparison of MXFP4 codes and E8M0 scales.  Mismatches are allowed only
     where the fp32 pre-rounding value (oracle V) lies within 1 ulp of a rounding boundary
-    (or the block max within 1 ulp of a power of two); those are counted and returned."""
+    (or the block max within 1 ulp of a power of two); those are counted and returned, and
+    recorded under `label` for the session summary.  V may be a callable that returns it
+    (computed only when there is a mismatch)."""
     gs = layout.tiled_to_rowmajor(gpu_scales_tiled, rows, K)
     pad = layout.padded_block_bytes(gpu_scales_tiled, rows, K)
     assert np.all(pad == 0), "padded scale blocks of real rows must be zero"
@@ -53,9 +75,13 @@ def compare_mx(gpu_codes, gpu_scales_tiled, ref_codes, ref_scales, rows, K, V=No
     gn = unpack_nibbles(gpu_codes)
     rn = unpack_nibbles(ref_codes)
     bad_c = gn != rn
-    stats = {"code_mismatch": int(bad_c.sum()), "scale_mismatch": int(bad_s.sum()), "exempt": 0}
+    stats = {"codes": int(bad_c.size), "scales": int(bad_s.size), "code_mismatch": int(bad_c.sum()),
+             "scale_mismatch": int(bad_s.sum()), "exempt": 0}
     if not bad_c.any() and not bad_s.any():
+        _record(label, stats)
         return stats
+    if callable(V):
+        V = V()
     assert V is not None, f"mismatches without oracle values: {stats}"
     Vb = V.reshape(rows, K // 32, 32)
     amax = np.abs(Vb).max(-1)
@@ -64,6 +90,7 @@ def compare_mx(gpu_codes, gpu_scales_tiled, ref_codes, ref_scales, rows, K, V=No
     ok_c = ~bad_c | _near_code_boundary(V, e_full) | np.repeat(bad_s & ok_s, 32, axis=1)
     stats["exempt"] = int((bad_c & ok_c).sum() + (bad_s & ok_s).sum())
     assert ok_s.all() and ok_c.all(), f"non-exempt mismatches: {stats}"
+    _record(label, stats)
     return stats
 
 

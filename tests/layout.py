@@ -36,3 +36,15 @@ def padded_block_bytes(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
     kbp = padded_blocks(K)
     idx = scale_index(rows, K, kbp)[:, K // 32:]
     return np.asarray(buf)[idx]
+
+
+def rows_of_tiled(buf: np.ndarray, rows, K: int) -> np.ndarray:
+    """A scale buffer in the same layout holding only the listed rows (in that order), padded
+    blocks included, so a sample of rows can be compared like a whole matrix."""
+    kbp = padded_blocks(K)
+    r = np.asarray(rows, dtype=np.int64)[:, None]
+    kb = np.arange(kbp, dtype=np.int64)[None, :]
+    src = ((r // 128) * (kbp // 4) + kb // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + kb % 4
+    out = np.zeros(scale_bytes(len(rows), K), np.uint8)
+    out[scale_index(len(rows), K, kbp)] = np.asarray(buf)[src]
+    return out

@@ -65,3 +65,39 @@ def test_reference_arm_prints_only_on_rank_zero(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(None)  # rank 1 returns before touching its arguments
     assert buf.getvalue() == ""
+
+
+def test_summary_and_mx_diff_on_fake_results():
+    """The bench's end-of-line summary reads every leg's figures (a missing key would end a long
+    GPU run without its line), and its code comparison counts mismatches and exempt ones."""
+    import numpy as np
+
+    import bench
+    lr = {"frac": 0.6}
+    leg = {"roofline": {"frac": 0.7}, "overhead": {"vs_plain_mxfp4_pct": 3.0, "vs_gemm_only_pct": 9.0}}
+    out = {"value": 4000.0, "linear_roofline": lr, **leg,
+           "secondary": {"llama3_8b_up_prefill": {"tflops": 4000.0, "linear_roofline": lr, **leg},
+                         "qwen3_32b_up_decode_M1": {"gbs": 3600.0, "linear_roofline": lr, "vs_plain_mxfp4_pct": 2.0},
+                         "qwen3_32b_stack": {"layers": 64, "M1": {"w4a4_ms": 6.5, "linear_roofline_frac": 0.4,
+                                                                  "vs_plain_mxfp4_pct": 3.0}},
+                         "qwen3_moe_grouped": {"experts": 128, "up_T16": {"ms": 0.015, "linear_roofline_frac": 0.5,
+                                                                          "vs_plain_mxfp4_pct": 3.0}}},
+           "parity": {"ok": True, "activations": {"exempt": 0}, "weights": {"exempt": 0}, "y_rel_fro_vs_oracle": 1e-6}}
+    sm = bench.summary(out)
+    assert set(sm) == {"cfg4_down_prefill", "cfg2_llama_up", "cfg3_M1", "cfg5_M1", "moe_up_T16", "parity_cfg4"}
+    codes = np.zeros((1, 16), np.uint8)  # one 32-element block
+    codes[0, :2] = [0x21, 0x43]
+    scales = np.array([[120]], np.uint8)
+    V = np.zeros((1, 32), np.float32)
+    V[0, :4] = [2.0 ** -8, 2.0 ** -7, 1.5 * 2.0 ** -7, 2.0 ** -6]
+    same = bench._mx_diff(codes, scales, codes.copy(), scales.copy(), V)
+    assert same == {"codes": 32, "code_mismatch": 0, "scales": 1, "scale_mismatch": 0, "exempt": 0}
+    # element 1 differs; the oracle's value 2^-7 at scale 2^(120-127) is 1.0 on the E2M1 grid, not
+    # near a rounding boundary, so the mismatch is not exempt
+    other = codes.copy()
+    other[0, 0] = 0x31
+    diff = bench._mx_diff(other, scales, codes, scales, V)
+    assert diff["code_mismatch"] == 1 and diff["exempt"] == 0
+    # a value exactly on the 1.25 boundary (scaled) is exempt
+    V[0, 1] = 1.25 * 2.0 ** -7
+    assert bench._mx_diff(other, scales, codes, scales, V)["exempt"] == 1

@@ -52,6 +52,68 @@ def test_linear_end_to_end(mq, wl):
     assert err <= 1e-3
 
 
+# The 64-layer Qwen3-32B-shaped stack: every linear shape of a decoder layer (each from a
+# different layer, so different seeds) at every token count of the stack sweep.  Each layer is
+# its own problem ("MACaQ", Abstract: every linear layer is treated independently), with its own
+# calibrated scale, fold and multipliers.
+STACK_LAYER_OF = {"q": 5, "k": 17, "v": 29, "o": 40, "gate": 51, "up": 58, "down": 63}
+
+
+@pytest.fixture(scope="module")
+def stack_folds(mq):
+    """Per stack linear (built once, reused for every M): s, the GPU fold and the oracle fold;
+    the GPU fold is checked against the oracle's bit for bit on the way."""
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            wl = wls.stack_layer(STACK_LAYER_OF[name], name, 1)
+            W = wls.make_w(wl)
+            s = wls.make_s(wl, W)
+            Wq, Ws, am = mq.macaq_fold_weights(W.cuda(), s.cuda())
+            torch.cuda.synchronize()
+            Wf = W.numpy()
+            del W
+            rWq, rWs, ra = oracle.fold_weights(Wf, s.numpy())
+            assert np.array_equal(gu.to_np(am).view(np.uint32), ra.view(np.uint32))
+            _, w = oracle.multipliers(s.numpy())
+            gu.compare_mx(gu.to_np(Wq), gu.to_np(Ws), rWq, rWs, wl.N, wl.K, lambda: oracle.transform_f32(Wf, w),
+                          label=gu.config_label(wl, "fold"))
+            cache[name] = (Wq, Ws, am, rWq, rWs, ra)
+        return cache[name]
+
+    return get
+
+
+@pytest.mark.parametrize("M", wls.STACK_M)
+@pytest.mark.parametrize("name", list(STACK_LAYER_OF))
+def test_stack_linear_matches_oracle(mq, stack_folds, name, M):
+    """One linear of the stack at one token count, in the launch configuration the stack sweep
+    times (the linear with a caller workspace): activation codes and scales of sampled rows bit
+    for bit (near-boundary mismatches counted), y of those rows within the GEMM tolerance of
+    the oracle's contraction of its own codes."""
+    wl = wls.stack_layer(STACK_LAYER_OF[name], name, M)
+    Wq, Ws, am, rWq, rWs, ra = stack_folds(name)
+    x = wls.make_x(wl)
+    xd = x.cuda()
+    ws = torch.full((mq.linear_workspace_bytes(M, wl.N, wl.K),), 0xA5, dtype=torch.uint8, device="cuda")
+    y = mq.macaq_w4a4_linear(xd, am, Wq, Ws, wl.N, workspace=ws)
+    Aq, As = mq.macaq_act_transform_quant(xd, am)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status() == 0
+    rng = np.random.default_rng(7 * M + wl.layer)
+    rows = np.arange(M) if M <= 64 else np.unique(np.r_[0, M - 1, rng.choice(M, 22, replace=False)])
+    xf = x.float().numpy()[rows]
+    V = oracle.transform_f32(xf, ra)
+    rAq, rAs = oracle.quantize_mx(V)
+    gAs = layout.rows_of_tiled(gu.to_np(As), rows, wl.K)
+    gu.compare_mx(gu.to_np(Aq)[rows], gAs, rAq, rAs, len(rows), wl.K, V, label=gu.config_label(wl, "act"))
+    ref = oracle.mx_gemm(rAq, rAs, rWq, rWs)
+    err = gu.rel_fro(gu.to_np(y.float())[rows], gu.bf16_round(ref))
+    print(f"stack {name} M={M}: {len(rows)} rows vs oracle {err:.2e}")
+    assert err <= 1e-3
+
+
 def test_linear_zero_input_gives_zero(mq):
     M, K, N = 5, 256, 384
     W = torch.randn(N, K, device="cuda") * 0.02

@@ -48,7 +48,7 @@ def test_act_transform_quant_matches_oracle(mq, wl):
     xf = x.float().numpy()
     V = oracle.transform_f32(xf, a)
     rc, rs = oracle.quantize_mx(V)
-    stats = gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, wl.M, wl.K, V)
+    stats = gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, wl.M, wl.K, V, label=gu.config_label(wl, "act"))
     print(wl.name, wl.M, stats)
 
 
@@ -70,9 +70,9 @@ def test_act_quant_large_ragged(mq, M, K):
     xf = xb.float().numpy()
     V = oracle.transform_f32(xf, a)
     rc, rs = oracle.quantize_mx(V)
-    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, M, K, V)
+    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, M, K, V, label="large ragged act")
     pc, ps = oracle.quantize_mx(xf)
-    gu.compare_mx(gu.to_np(Pq), gu.to_np(Ps), pc, ps, M, K, xf)
+    gu.compare_mx(gu.to_np(Pq), gu.to_np(Ps), pc, ps, M, K, xf, label="large ragged plain")
 
 
 @pytest.mark.parametrize("wl", [wls.TINY, wls.LLAMA_UP, wls.QWEN_DOWN], ids=lambda w: w.name)
@@ -82,7 +82,7 @@ def test_act_quant_plain_matches_oracle(mq, wl):
     torch.cuda.synchronize()
     xf = x.float().numpy()
     rc, rs = oracle.act_quant_plain(xf)
-    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, wl.M, wl.K, xf)
+    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, wl.M, wl.K, xf, label=gu.config_label(wl, "plain"))
 
 
 @pytest.mark.parametrize("wl", [wls.TINY, wls.LLAMA_UP, wls.QWEN_UP_DECODE, wls.QWEN_DOWN], ids=lambda w: w.name)
@@ -95,7 +95,7 @@ def test_fold_weights_matches_oracle(mq, wl):
     assert np.array_equal(gu.to_np(am).view(np.uint32), a.view(np.uint32))
     V = oracle.transform_f32(W.numpy(), w)
     rc, rs = oracle.quantize_mx(V)
-    stats = gu.compare_mx(gu.to_np(Wq), gu.to_np(Ws), rc, rs, wl.N, wl.K, V)
+    stats = gu.compare_mx(gu.to_np(Wq), gu.to_np(Ws), rc, rs, wl.N, wl.K, V, label=gu.config_label(wl, "fold"))
     print(wl.name, stats)
 
 
@@ -131,9 +131,9 @@ def test_act_transform_quant_edge_cases(mq, name, x):
     xf = xb.float().numpy()
     V = oracle.transform_f32(xf, a)
     rc, rs = oracle.quantize_mx(V)
-    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, M, K, V)
+    gu.compare_mx(gu.to_np(Aq), gu.to_np(As), rc, rs, M, K, V, label="edge cases act")
     pc, ps = oracle.quantize_mx(xf)
-    gu.compare_mx(gu.to_np(Pq), gu.to_np(Ps), pc, ps, M, K, xf)
+    gu.compare_mx(gu.to_np(Pq), gu.to_np(Ps), pc, ps, M, K, xf, label="edge cases plain")
 
 
 def test_fold_rejects_invalid_scale(mq):

@@ -6,7 +6,8 @@ scratch in a static 32 MiB device array of the library instead of a caller works
 Called here through the C ABI (ctypes, raw device pointers) and compared with
 macaq_w4a4_linear on two calls in a row -- a larger problem, then a smaller one, so the
 second runs over the first one's leftover scratch -- within the GEMM tolerance of the other
-tests.  This file is collected last so a stop-at-first-failure run has run the rest first."""
+tests; and, on a problem too large for the GEMM's stream-K scratch to fit beside the
+activations, with the oracle and with the data-parallel GEMM it falls back to.  This file is collected last so a stop-at-first-failure run has run the rest first."""
 import ctypes
 
 import numpy as np
@@ -64,6 +65,38 @@ def test_noalloc_matches_linear_on_two_calls_in_a_row(mq):
     assert _rel(y2, r2) <= TOL
     assert torch.count_nonzero(r1).item() > 0 and torch.count_nonzero(r2).item() > 0
     assert mq.macaq_device_status() == 0
+
+
+def test_noalloc_against_oracle_and_its_data_parallel_fallback(mq):
+    """A problem whose activation codes and scales fit the 32 MiB array but whose whole
+    workspace (with the GEMM's stream-K scratch) does not: the GEMM then runs its
+    data-parallel schedule, so the output equals, bit for bit, the data-parallel GEMM of the
+    same codes.  Called right after a smaller stream-K problem, so it runs over that call's
+    leftover scratch, and checked on sampled rows against the oracle's own fold,
+    quantisation and fp64 contraction."""
+    import oracle
+    from tests import gpu_util as gu
+    M, K, N = 4096, 8192, 2560
+    act = M * K // 2 + mq.scale_bytes(M, K)
+    assert act <= mq.NOALLOC_SCRATCH_BYTES < mq.linear_workspace_bytes(M, N, K)
+    small = _layer(mq, 200, 1024, 768, 3)
+    _noalloc_via_c_abi(mq, small[0], small[3], small[1], small[2], 768)
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    W = torch.randn(N, K, generator=g) * 0.02
+    s = torch.rand(K, generator=g) * 4 + 0.25
+    Wq, Ws, am = mq.macaq_fold_weights(W.cuda(), s.cuda())
+    y = _noalloc_via_c_abi(mq, x.cuda(), am, Wq, Ws, N)
+    Aq, As = mq.macaq_act_transform_quant(x.cuda(), am)
+    dp = mq.macaq_mxfp4_gemm(Aq, As, Wq, Ws, M, N, K, data_parallel=True)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status() == 0
+    assert torch.equal(y, dp)
+    rows = np.sort(np.random.default_rng(5).choice(M, 16, replace=False))
+    rWq, rWs, ra = oracle.fold_weights(W.numpy(), s.numpy())
+    rAq, rAs = oracle.act_transform_quant(x.float().numpy()[rows], ra)
+    ref = oracle.mx_gemm(rAq, rAs, rWq, rWs)
+    assert gu.rel_fro(gu.to_np(y.float())[rows], gu.bf16_round(ref)) <= TOL
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(mq):
