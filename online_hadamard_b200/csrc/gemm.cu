@@ -102,6 +102,7 @@ struct GemmParams {
     int64_t ldy;          // elements per row of y
     int y_fp32;
     int num_p_tiles, num_q_tiles, num_k_tiles, q_row_blocks;
+    int raster_group;     // pair kernel: activation panels per group of the tile order (pair_tile)
     int dp_tiles;         // tiles scheduled data-parallel (blockIdx.x + i * gridDim.x)
     int64_t sk_units;     // K steps of the remaining tiles, split evenly over the first sk_count units
     int sk_count;         // scheduling units that take part in the split (<= the units launched)
@@ -730,6 +731,23 @@ struct PairCfg {
     static_assert(kSFBase + kPairStages * kSFBufCols <= kTmemCols, "tensor memory budget");
 };
 
+// Order of the pair kernel's 256 x 256 tiles: groups of `raster_group` activation panels (256
+// rows each), the last group possibly smaller; within a group the weight panel varies slowest
+// and the activation panel fastest.  A wave of consecutive tiles then touches about
+// raster_group activation panels and (pairs / raster_group) weight panels, and a group's
+// activation panels are reused from L2 across the waves that sweep the weight panels, instead
+// of every wave streaming the whole weight matrix again (activation-major order: each wave
+// touches every weight panel).  Tile numbers past dp_tiles (stream-K) follow the same order.
+__device__ __forceinline__ void pair_tile(const GemmParams& prm, int tile, int& pt, int& qt) {
+    const int per_group = prm.raster_group * prm.num_q_tiles;
+    const int g = tile / per_group;
+    const int local = tile - g * per_group;
+    const int first = g * prm.raster_group;
+    const int rows = prm.num_p_tiles - first < prm.raster_group ? prm.num_p_tiles - first : prm.raster_group;
+    pt = first + local % rows;
+    qt = local / rows;
+}
+
 template <int STAGES>
 __global__ void __launch_bounds__(kPairThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -791,8 +809,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             WorkIter it(prm, pair, pairs);
             Work w;
             while (!abort && it.next(prm, w)) {
-                const int pt = w.tile / prm.num_q_tiles;  // activation-block major: early tiles need early rows
-                const int qt = w.tile % prm.num_q_tiles;
+                int pt, qt;
+                pair_tile(prm, w.tile, pt, qt);
                 const int a_row = pt * 256 + static_cast<int>(rank) * 128;
                 const int b_row = qt * 256 + static_cast<int>(rank) * 128;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
@@ -907,8 +925,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         WorkIter it(prm, pair, pairs);
         Work w;
         while (!abort && it.next(prm, w)) {
-            const int pt = w.tile / prm.num_q_tiles;  // activation-block major: early tiles need early rows
-            const int qt = w.tile % prm.num_q_tiles;
+            int pt, qt;
+            pair_tile(prm, w.tile, pt, qt);
             if (!mbar_wait(acc_full, acc_phase, &abort)) break;
             acc_phase ^= 1u;
             tc_fence_after();
@@ -1270,6 +1288,14 @@ static int gemm_pairs_query() {
     return clusters;
 }
 
+// Activation panels per group of the pair kernel's tile order: a wave of `pairs` tiles touches
+// about g activation and pairs / g weight panels (equal sizes), fewest near g = sqrt(pairs).
+static int pair_raster_group(int p_tiles, int pairs) {
+    int g = 1;
+    while ((g + 1) * (g + 1) <= pairs) ++g;
+    return g < p_tiles ? g : p_tiles;
+}
+
 static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int pairs, cudaStream_t stream, bool pdl) {
     CUtensorMap ma, mb, msa, msb, my;
     if (!make_codes_map(&ma, op.pq, op.p_rows, op.K, 128) || !make_codes_map(&mb, op.qq, op.q_rows, op.K, 128) ||
@@ -1289,6 +1315,7 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     prm.num_q_tiles = static_cast<int>((op.q_rows + 255) / 256);
     prm.num_k_tiles = static_cast<int>((op.K + kStageK - 1) / kStageK);
     prm.q_row_blocks = static_cast<int>((op.q_rows + 127) / 128);
+    prm.raster_group = pair_raster_group(prm.num_p_tiles, pairs);
     prm.tma_store = (!op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
     if (prm.tma_store && !make_out_map(&my, op.y, op.p_rows, op.q_rows, op.ldy)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = ma;  // unused placeholder

@@ -52,12 +52,13 @@ def test_act_transform_quant_matches_oracle(mq, wl):
     print(wl.name, wl.M, stats)
 
 
-@pytest.mark.parametrize("M,K", [(1037, 4128), (4099, 1056), (64, 65600)], ids=lambda v: str(v))
+@pytest.mark.parametrize("M,K", [(1037, 4128), (4099, 1056), (64, 65600), (4099, 4128)], ids=lambda v: str(v))
 def test_act_quant_large_ragged(mq, M, K):
     """Inputs above the small-input size, so the whole-block kernel (one thread per 32-element
-    block, rows walked two at a time) runs, with row counts that leave a thread an odd last row
-    and K that is not a multiple of 256 (padded scale blocks): transform and plain codes
-    against the oracle."""
+    block, rows walked two at a time, or one row ahead for transforms of 16 M elements and
+    more: the last case) runs, with row counts that leave a thread an odd last row and K that
+    is not a multiple of 256 (padded scale blocks): transform and plain codes against the
+    oracle."""
     assert M * K > (1 << 22)
     rng = np.random.default_rng(M + K)
     xf32 = rng.standard_t(4, (M, K)).astype(np.float32) * rng.uniform(0.1, 30.0, (1, K)).astype(np.float32)
