@@ -19,6 +19,12 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB_PATH = os.path.join(BUILD_DIR, "libmacaq.so")
+# Fault-injection build for the tests only: stream-K owners give up on a flag after 200 000 cycles
+# (~0.1 ms) instead of ~4 s, and macaq_test_owner_tag_offset() can make them wait for a tag that no
+# contributor writes, so a test can see a bounded device-side wait run out.  Never loaded by the
+# product path.
+FAULT_LIB_PATH = os.path.join(BUILD_DIR, "libmacaq_faultwait.so")
+FAULT_FLAGS = ["-DMACAQ_TEST_HOOKS", "-DMACAQ_FLAG_WAIT_LIMIT=200000"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -40,28 +46,35 @@ def _sources() -> list[str]:
                   + [os.path.join(INCLUDE, "macaq.h")])
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def is_stale(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    if not force and not is_stale():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          path: str = LIB_PATH) -> str:
+    if not force and not is_stale(path):
+        return path
     os.makedirs(BUILD_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    tmp = path + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
            "-o", tmp, os.path.join(CSRC, "libmacaq.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
+
+
+def build_fault_library(force: bool = False) -> str:
+    """The fault-injection build (tests only), next to the product library."""
+    return build(force=force, extra_flags=FAULT_FLAGS, path=FAULT_LIB_PATH)
 
 
 if __name__ == "__main__":
     v = "-v" in sys.argv
     flags = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None
     print(build(force=True, verbose=v, extra_flags=flags))
+    print(build_fault_library(force=True))

@@ -110,6 +110,7 @@ struct GemmParams {
     float* partials;      // stream-K fp32 partial accumulators, one 128 x BN slot per CTA
     uint64_t* flags;      // stream-K hand-off: one word per (partial slot, epilogue thread)
     uint64_t tag;         // this launch's value of a written flag word (unique per launch)
+    uint64_t owner_tag;   // the value an owner waits for: tag (a fault-injection build can shift it)
     int tma_store;        // bf16 output written by TMA from shared memory (non-swap, N % 8 == 0)
 };
 
@@ -233,6 +234,23 @@ struct WorkIter {
     }
 };
 
+// Bound of an owner's wait for a contributor's stream-K flag.  A fault-injection build of the
+// library (MACAQ_TEST_HOOKS, tests only) shortens it, so a test can make the wait run out: the
+// owner then records MACAQ_ETIMEOUT in the device status and finishes its item.
+#ifdef MACAQ_FLAG_WAIT_LIMIT
+constexpr long long kFlagWaitLimitCycles = MACAQ_FLAG_WAIT_LIMIT;
+#else
+constexpr long long kFlagWaitLimitCycles = kWaitLimitCycles;
+#endif
+
+#ifdef MACAQ_TEST_HOOKS
+// Added to the tag owners wait for (0: none): with 1 no contributor ever writes the awaited value.
+static std::atomic<int64_t> g_test_owner_tag_offset{0};
+static uint64_t owner_tag_of(uint64_t tag) { return tag + static_cast<uint64_t>(g_test_owner_tag_offset.load()); }
+#else
+static uint64_t owner_tag_of(uint64_t tag) { return tag; }
+#endif
+
 __device__ __forceinline__ uint64_t ld_acquire64(const uint64_t* p) {
     uint64_t v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -276,8 +294,8 @@ __device__ __forceinline__ void sum_partials(const GemmParams& prm, const Work& 
         uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + etid;
         if (!abort) {
             const long long t0 = clock64();
-            while (ld_acquire64(flag) != prm.tag) {
-                if (clock64() - t0 > kWaitLimitCycles) {
+            while (ld_acquire64(flag) != prm.owner_tag) {
+                if (clock64() - t0 > kFlagWaitLimitCycles) {
                     atomicExch(&g_device_status, MACAQ_ETIMEOUT);
                     abort = 1;
                     break;
@@ -327,8 +345,8 @@ __device__ __forceinline__ void finish_item(const GemmParams& prm, const CUtenso
             uint64_t* flag = prm.flags + static_cast<int64_t>(slot_id) * kEpiThreads + e.etid;
             if (!abort) {
                 const long long t0 = clock64();
-                while (ld_acquire64(flag) != prm.tag) {
-                    if (clock64() - t0 > kWaitLimitCycles) {
+                while (ld_acquire64(flag) != prm.owner_tag) {
+                    if (clock64() - t0 > kFlagWaitLimitCycles) {
                         atomicExch(&g_device_status, MACAQ_ETIMEOUT);
                         abort = 1;
                         break;
@@ -1220,6 +1238,7 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
         prm.flags = static_cast<uint64_t*>(ws.ptr);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + streamk_flag_bytes(ctas));
         prm.tag = next_launch_tag();
+        prm.owner_tag = owner_tag_of(prm.tag);
     }
 
     cudaLaunchConfig_t cfg = {};
@@ -1334,6 +1353,7 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
         prm.flags = static_cast<uint64_t*>(ws.ptr);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws.ptr) + streamk_flag_bytes(ctas));
         prm.tag = next_launch_tag();
+        prm.owner_tag = owner_tag_of(prm.tag);
     }
 
     cudaLaunchConfig_t cfg = {};
@@ -1567,3 +1587,8 @@ extern "C" int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* count
     const GemmOperands op{Aq, As, Wq, Ws, P, E * N, K, y, N, 0};
     return launch_gemm<256, 4, false, true>(op, none, st, true, &gt, N);
 }
+
+#ifdef MACAQ_TEST_HOOKS
+// Fault injection (test build only): offset of the tag stream-K owners wait for.
+extern "C" void macaq_test_owner_tag_offset(int64_t offset) { macaq::g_test_owner_tag_offset.store(offset); }
+#endif

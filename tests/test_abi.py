@@ -175,3 +175,14 @@ def test_binding_refuses_a_stream_of_another_device():
         mq._check_stream_device(types.SimpleNamespace(device=torch.device("cpu")), dev0)
     mq._check_stream_device(types.SimpleNamespace(device=torch.device("cuda", 0)), dev0)
     mq._check_stream_device(types.SimpleNamespace(device="cuda:0"), dev0)
+
+
+def test_fault_injection_hook_only_in_the_test_build():
+    """The tag-offset hook exists only in the fault-injection build that one GPU test loads; the
+    product library does not export it."""
+    import ctypes
+
+    from online_hadamard_b200 import build as b
+    fault = ctypes.CDLL(b.build_fault_library())
+    assert hasattr(fault, "macaq_test_owner_tag_offset")
+    assert not hasattr(mq.load_library(), "macaq_test_owner_tag_offset")
