@@ -69,6 +69,8 @@ def _load():
             lib.oracle_mx_decode.argtypes = [p, p, i64, i64, p]
             lib.oracle_mx_gemm.argtypes = [p, p, p, i64, p, p, i64, i64, p]
             lib.oracle_calibrate_scale.argtypes = [p, i64, p, i64, i64, p]
+            lib.oracle_hessian.argtypes = [p, i64, i64, p]
+            lib.oracle_flip_refine.argtypes = [p, i64, i64, p, p, p, i64, p]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -215,6 +217,49 @@ def calibrate_scale(xcal, W) -> np.ndarray:
     s = np.empty(K, np.float32)
     _load().oracle_calibrate_scale(_ptr(xcal), C, _ptr(W), N, K, _ptr(s))
     return s
+
+
+def hessian_of(Xt) -> np.ndarray:
+    """Hs = Xt^T Xt (fp64 [K][K]) of transformed calibration activations Xt [C][K] (fp32),
+    each entry an fma chain over the calibration rows in order (Flip-Refinement)."""
+    Xt = _f32(Xt)
+    C, K = Xt.shape
+    Hs = np.empty((K, K), np.float64)
+    _load().oracle_hessian(_ptr(Xt), C, K, _ptr(Hs))
+    return Hs
+
+
+def calib_hessian(xcal, act_mult) -> np.ndarray:
+    """Hs of a calibration batch xcal [C][K] (bf16 values): the online transform with the layer's
+    activation multipliers, then Xt^T Xt in fp64."""
+    return hessian_of(transform_f32(xcal, act_mult))
+
+
+def flip_refine_codes(V, codes, scales, Hs, max_moves) -> tuple[np.ndarray, np.ndarray]:
+    """Flip-Refinement (see macaq_oracle.c) of round-to-nearest codes [N][K/2] of the folded
+    weights V [N][K] (fp32) with their E8M0 scales [N][K/32] kept: (refined codes, moves per row)."""
+    V = _f32(V)
+    N, K = V.shape
+    _check_k(K)
+    out = np.array(codes, dtype=np.uint8, copy=True, order="C")
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    Hs = np.ascontiguousarray(Hs, dtype=np.float64)
+    if Hs.shape != (K, K) or out.shape != (N, K // 2) or scales.shape != (N, K // 32):
+        raise ValueError("shape mismatch")
+    moves = np.empty(N, np.int64)
+    _load().oracle_flip_refine(_ptr(V), N, K, _ptr(Hs), _ptr(out), _ptr(scales), int(max_moves), _ptr(moves))
+    return out, moves
+
+
+def flip_refine(W, s, xcal, max_moves) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The whole offline step for one layer: fold W with s (round-to-nearest codes), Hessian of the
+    transformed calibration batch, Flip-Refinement.  Returns (codes, scales, moves per row)."""
+    a, w = multipliers(s)
+    V = transform_f32(W, w)
+    codes, scales = quantize_mx(V)
+    Hs = calib_hessian(xcal, a)
+    refined, moves = flip_refine_codes(V, codes, scales, Hs, max_moves)
+    return refined, scales, moves
 
 
 def num_threads() -> int:

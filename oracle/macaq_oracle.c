@@ -240,6 +240,116 @@ void oracle_mx_gemm(const uint8_t* Aq, const uint8_t* As, const int64_t* rows, i
     free(a);
 }
 
+/* ------------------------------------------------------------------ Flip-Refinement
+ *
+ * "MACaQ ...", Abstract: to improve over round-to-nearest, Flip-Refinement is a Hessian-aware
+ * coordinate-descent procedure that greedily moves individual FP4 codes to adjacent representable
+ * values (the French news page adds: in place of GPTQ-style updates).  The pages give no more;
+ * the readings used here:
+ *   - it refines one layer's folded weight codes W' = MXFP4(W diag(w) H_bd), starting from the
+ *     round-to-nearest codes, with every E8M0 block scale kept (only codes move);
+ *   - the objective of output row n is the layer's output error on the calibration batch,
+ *       L_n = (q_n - v_n) Hs (q_n - v_n)^T,   Hs = Xt^T Xt,
+ *     q_n the decoded refined row, v_n the fp32 folded row before quantisation, and Xt the
+ *     calibration activations after the online transform (fp32, before their quantisation);
+ *   - "adjacent representable values": the 15 distinct E2M1 values -6 .. 6 in order; a move
+ *     takes one code one step up or down that line (at +-6 only inwards); a code that moves to
+ *     zero keeps its sign bit;
+ *   - "greedily": each step applies, in one row, the single move with the most negative change
+ *     dL = d (2 g_k + d Hs_kk) (g = Hs r, r = q - v, d the value step times the block scale);
+ *     ties go to the smaller k, then to the downward move; a row stops when no move lowers L or
+ *     after max_moves moves.
+ * Arithmetic (fp64, one order, so another implementation can reproduce every decision):
+ *   Hs[j][k] = sum over calibration rows c ascending of Xt[c][j] Xt[c][k], as fma(Xt, Xt, acc)
+ *   from +0; r_k = q_k - v_k; g_j = sum over k ascending of Hs[j][k] r_k as fma from +0;
+ *   dL = d * fma(d, Hs[k][k], 2 g_k); after a move of coordinate k by d:
+ *   g_j = fma(d, Hs[j][k], g_j) for every j, r_k = r_k + d. */
+
+/* Hs = Xt^T Xt for transformed calibration activations Xt [C][K] (fp32), fp64 [K][K]. */
+void oracle_hessian(const float* Xt, int64_t C, int64_t K, double* Hs) {
+#pragma omp parallel for schedule(dynamic, 8)
+    for (int64_t j = 0; j < K; ++j) {
+        for (int64_t k = 0; k < K; ++k) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < C; ++c) acc = fma((double)Xt[c * K + j], (double)Xt[c * K + k], acc);
+            Hs[j * K + k] = acc;
+        }
+    }
+}
+
+/* The 15 E2M1 values in increasing order; position 7 is zero. */
+static const double kE2M1Line[15] = {-6.0, -4.0, -3.0, -2.0, -1.5, -1.0, -0.5, 0.0,
+                                     0.5,  1.0,  1.5,  2.0,  3.0,  4.0,  6.0};
+
+/* Position of a 4-bit code on that line (both zero codes sit at 7). */
+static int e2m1_line_pos(int code) {
+    const int m = code & 7;
+    return (code & 8) ? 7 - m : 7 + m;
+}
+
+/* Code of line position p; a zero keeps the sign bit of `old`. */
+static int e2m1_code_at(int p, int old) {
+    if (p == 7) return old & 8;
+    return p > 7 ? p - 7 : 8 | (7 - p);
+}
+
+/* Flip-Refinement of weight codes in place.  V [N][K] fp32 folded weights before quantisation,
+ * codes [N][K/2] (their round-to-nearest codes on entry), scales [N][K/32] E8M0 (unchanged),
+ * Hs [K][K].  moves[n] = the moves applied to row n. */
+void oracle_flip_refine(const float* V, int64_t N, int64_t K, const double* Hs, uint8_t* codes,
+                        const uint8_t* scales, int64_t max_moves, int64_t* moves) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; ++n) {
+        int* c = (int*)malloc(sizeof(int) * K);
+        double* unit = (double*)malloc(sizeof(double) * K);
+        double* r = (double*)malloc(sizeof(double) * K);
+        double* g = (double*)malloc(sizeof(double) * K);
+        for (int64_t k = 0; k < K; ++k) {
+            const uint8_t byte = codes[n * (K / 2) + k / 2];
+            c[k] = (k & 1) ? byte >> 4 : byte & 15;
+            unit[k] = ldexp(1.0, (int)scales[n * (K / 32) + k / 32] - 127);
+            r[k] = kE2M1Line[e2m1_line_pos(c[k])] * unit[k] - (double)V[n * K + k];
+        }
+        for (int64_t j = 0; j < K; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc = fma(Hs[j * K + k], r[k], acc);
+            g[j] = acc;
+        }
+        int64_t done = 0;
+        while (done < max_moves) {
+            double best = 0.0;
+            int64_t bk = -1;
+            int bp = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                const int p = e2m1_line_pos(c[k]);
+                for (int dir = -1; dir <= 1; dir += 2) {
+                    const int q = p + dir;
+                    if (q < 0 || q > 14) continue;
+                    const double d = (kE2M1Line[q] - kE2M1Line[p]) * unit[k];
+                    const double dl = d * fma(d, Hs[k * K + k], 2.0 * g[k]);
+                    if (dl < best) {  /* strictly: ties keep the earlier candidate */
+                        best = dl;
+                        bk = k;
+                        bp = q;
+                    }
+                }
+            }
+            if (bk < 0) break;  /* no move lowers the objective */
+            const double d = (kE2M1Line[bp] - kE2M1Line[e2m1_line_pos(c[bk])]) * unit[bk];
+            c[bk] = e2m1_code_at(bp, c[bk]);
+            r[bk] = r[bk] + d;
+            for (int64_t j = 0; j < K; ++j) g[j] = fma(d, Hs[j * K + bk], g[j]);
+            ++done;
+        }
+        for (int64_t k = 0; k < K; k += 2) codes[n * (K / 2) + k / 2] = (uint8_t)(c[k] | (c[k + 1] << 4));
+        moves[n] = done;
+        free(c);
+        free(unit);
+        free(r);
+        free(g);
+    }
+}
+
 /* Per-channel scale from a calibration batch xcal [C][K] (bf16 values held in fp32) and the
  * weights W [N][K]: column maxima of |.|, then sqrt of their quotient in double, rounded once to
  * fp32; 1 for a column whose activation or weight maximum is zero. */
