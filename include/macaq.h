@@ -234,6 +234,45 @@ int macaq_w4a4_linear_noalloc(const uint16_t* x, int64_t M, int64_t K, const flo
                               const uint8_t* Wq, const uint8_t* Ws, int64_t N, uint16_t* y,
                               void* stream);
 
+/*
+ * Flip-Refinement (Abstract: "a Hessian-aware coordinate-descent procedure that greedily moves
+ * individual FP4 codes to adjacent representable values", improving on round-to-nearest).  An
+ * offline step between macaq_fold_weights and inference; the pages give no more, and this library
+ * reads it as follows (details in csrc/flip.cu):
+ *   objective of weight row n:  L_n = (q_n - v_n) Hs (q_n - v_n)^T, q_n the decoded codes, v_n the
+ *   fp32 folded row before quantisation, Hs = Xt^T Xt with Xt a calibration batch after the online
+ *   transform; the E8M0 block scales stay as the fold set them; a move takes one code one step
+ *   along the ordered E2M1 values -6 .. 6 (a code reaching zero keeps its sign bit); each step
+ *   applies the row's single most-improving move (ties: smaller k, then downward); a row stops when
+ *   no move lowers L or after max_moves moves.  All of it in fp64 in one fixed order, so the
+ *   result is deterministic.
+ *
+ * macaq_calib_hessian -- Hs (fp64 [K][K], symmetric bit for bit) of a calibration batch.
+ *   xcal      in   bf16 bit patterns [C][K] (the layer's calibration activations)
+ *   act_mult  in   fp32 [K], the layer's multipliers (macaq_fold_weights)
+ *   Hs        out  fp64 [K][K] = Xt^T Xt, Xt[c][k] the fp32 online transform of xcal (scale and
+ *                  FWHT-32, as macaq_act_transform_quant computes it before quantising); each
+ *                  entry an fma chain over the calibration rows in order
+ *   workspace in   macaq_hessian_workspace_bytes(C, K) bytes (Xt, fp32)
+ * macaq_flip_refine -- refine folded weight codes in place.
+ *   W, s      in   the layer's fp32 weights [N][K] and per-channel scale [K] (as given to
+ *                  macaq_fold_weights)
+ *   Hs        in   from macaq_calib_hessian
+ *   Wq        in/out  round-to-nearest codes [N][K/2] from macaq_fold_weights; refined on return
+ *   Ws        in   their scales (unchanged)
+ *   max_moves in   moves per row at most (>= 0)
+ *   moves     out  int32 [N], moves applied per row (device; NULL: not reported)
+ *   workspace in   macaq_flip_refine_workspace_bytes(N, K) bytes
+ *   K <= 12288 (one row's state lives in shared memory), else MACAQ_ESHAPE.
+ */
+size_t macaq_hessian_workspace_bytes(int64_t C, int64_t K);
+int macaq_calib_hessian(const uint16_t* xcal, int64_t C, int64_t K, const float* act_mult, double* Hs,
+                        void* workspace, size_t workspace_bytes, void* stream);
+size_t macaq_flip_refine_workspace_bytes(int64_t N, int64_t K);
+int macaq_flip_refine(const float* W, int64_t N, int64_t K, const float* s, const double* Hs, uint8_t* Wq,
+                      const uint8_t* Ws, int64_t max_moves, int32_t* moves, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
 /* Sticky device-side status of the current device: MACAQ_OK, or MACAQ_ETIMEOUT once a
  * bounded wait inside a kernel gave up.  Synchronises the device.  `clear` != 0 resets it. */
 int macaq_device_status(int clear);

@@ -27,7 +27,7 @@ __all__ = [
     "load_library", "MacaqError", "scale_bytes", "scale_offset", "linear_workspace_bytes", "gemm_workspace_bytes",
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_grouped_linear",
-    "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc",
+    "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian", "macaq_flip_refine",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
@@ -38,6 +38,8 @@ EXPORTED_SYMBOLS = (
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_w4a4_linear",
     "macaq_act_quant_plain", "macaq_mxfp4_linear", "macaq_mxfp4_gemm", "macaq_device_status",
     "macaq_grouped_workspace_bytes", "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc",
+    "macaq_hessian_workspace_bytes", "macaq_calib_hessian", "macaq_flip_refine_workspace_bytes",
+    "macaq_flip_refine",
 )
 
 MACAQ_OK = 0
@@ -85,9 +87,16 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_w4a4_grouped_linear.argtypes = [p, p, i32, i64, p, p, p, i64, p, p, sz, p]
         lib.macaq_device_status.argtypes = [i32]
         lib.macaq_w4a4_linear_noalloc.argtypes = [p, i64, i64, p, p, p, i64, p, p]
+        lib.macaq_hessian_workspace_bytes.argtypes = [i64, i64]
+        lib.macaq_hessian_workspace_bytes.restype = sz
+        lib.macaq_calib_hessian.argtypes = [p, i64, i64, p, p, p, sz, p]
+        lib.macaq_flip_refine_workspace_bytes.argtypes = [i64, i64]
+        lib.macaq_flip_refine_workspace_bytes.restype = sz
+        lib.macaq_flip_refine.argtypes = [p, i64, i64, p, p, p, p, i64, p, p, sz, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
-                     "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc"):
+                     "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian",
+                     "macaq_flip_refine"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -368,6 +377,49 @@ def macaq_w4a4_linear_noalloc(x: torch.Tensor, act_mult: torch.Tensor, Wq: torch
         _check(load_library().macaq_w4a4_linear_noalloc(_ptr(x), M, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
                                                         _stream(stream, dev)), "macaq_w4a4_linear_noalloc")
     return y
+
+
+def macaq_calib_hessian(xcal: torch.Tensor, act_mult: torch.Tensor, Hs=None, workspace=None, stream=None):
+    """Hs = Xt^T Xt (fp64 [K, K]) of a bf16 calibration batch [C, K] after the online transform with
+    the layer's multipliers (Flip-Refinement's Hessian)."""
+    C, K = xcal.shape
+    _need(xcal, "xcal", torch.bfloat16)
+    dev = xcal.device
+    _need(act_mult, "act_mult", torch.float32, (K,), device=dev)
+    Hs = torch.empty(K, K, dtype=torch.float64, device=dev) if Hs is None else Hs
+    _need(Hs, "Hs", torch.float64, (K, K), device=dev)
+    need = int(load_library().macaq_hessian_workspace_bytes(C, K))
+    workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, min_numel=need, device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_calib_hessian(_ptr(xcal), C, K, _ptr(act_mult), _ptr(Hs), _ptr(workspace),
+                                                  workspace.numel(), _stream(stream, dev)), "macaq_calib_hessian")
+    return Hs
+
+
+def macaq_flip_refine(W: torch.Tensor, s: torch.Tensor, Hs: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor,
+                      max_moves: int, moves=None, workspace=None, stream=None):
+    """Flip-Refinement of the round-to-nearest codes Wq [N, K/2] (from macaq_fold_weights of W and s)
+    in place, scales Ws kept; returns the int32 moves applied per row."""
+    N, K = W.shape
+    _need(W, "W", torch.float32)
+    dev = W.device
+    _need(s, "s", torch.float32, (K,), device=dev)
+    _need(Hs, "Hs", torch.float64, (K, K), device=dev)
+    _need(Wq, "Wq", torch.uint8, (N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=scale_bytes(N, K), device=dev)
+    moves = torch.empty(N, dtype=torch.int32, device=dev) if moves is None else moves
+    _need(moves, "moves", torch.int32, (N,), device=dev)
+    need = int(load_library().macaq_flip_refine_workspace_bytes(N, K))
+    if need == 0:
+        raise ValueError(f"K={K} is not supported by macaq_flip_refine (K <= 12288, K % 32 == 0)")
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, min_numel=need, device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_flip_refine(_ptr(W), N, K, _ptr(s), _ptr(Hs), _ptr(Wq), _ptr(Ws), int(max_moves),
+                                                _ptr(moves), _ptr(workspace), workspace.numel(),
+                                                _stream(stream, dev)), "macaq_flip_refine")
+    return moves
 
 
 def macaq_device_status(clear: bool = False) -> int:
