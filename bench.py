@@ -530,8 +530,10 @@ def main():
     ms_e2e = max_over_ranks(time_eager(layer.e2e, e2e_steps, 3, device))
 
     extra = {}
+    if world > 1:
+        extra["tensor_parallel"] = tp_leg(mq, ranks, device, args)
     if not args.no_extra:
-        extra = secondary(mq, device, peaks, args)
+        extra.update(secondary(mq, device, peaks, args))
     if not args.no_stack:
         extra["qwen3_32b_stack"] = stack_sweep(mq, device, peaks)
         extra["qwen3_moe_grouped"] = moe_sweep(mq, device, peaks)
@@ -565,6 +567,37 @@ def main():
         out["summary"] = summary(out)
         print(json.dumps(out))
     ranks.close()
+
+
+def tp_leg(mq, ranks, device, args, wl=wls.QWEN_DOWN):
+    """The down projection split over the ranks by output columns (online_hadamard_b200.tensor_parallel):
+    each rank's W4A4 linear on its N / world weight rows, then the NCCL all-gather of the output
+    columns.  Eager launches timed with CUDA events, max over ranks; every rank takes the same
+    collective steps in warm-up and timing."""
+    from online_hadamard_b200 import tensor_parallel as tp
+    W = wls.make_w(wl)
+    s = wls.make_s(wl, W)
+    Wq, Ws, am = mq.macaq_fold_weights(W.to(device), s.to(device))
+    del W
+    q, sc, n = tp.shard_folded_weights(Wq, Ws, wl.N, wl.K, ranks.world, ranks.rank)
+    x = wls.make_x(wl).to(device)
+    ws = torch.empty(mq.linear_workspace_bytes(wl.M, max(n, 1), wl.K), dtype=torch.uint8, device=device)
+    step = lambda: tp.tp_w4a4_linear(x, am, q, sc, wl.N, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    ranks.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = ranks.max(e0.elapsed_time(e1) / args.steps)
+    ranks.barrier()
+    return {"workload": wl.name, "ranks": ranks.world, "rows_per_rank": n, "ms": ms,
+            "tflops": wl.flops / (ms * 1e-3) / 1e12, "scaling": "strong (one layer split over the ranks)",
+            "collective": "all-gather of the bf16 output columns"}
 
 
 def prefill_leg(layer, args, peaks):
