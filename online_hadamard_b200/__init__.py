@@ -28,6 +28,7 @@ __all__ = [
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_grouped_linear",
     "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian", "macaq_flip_refine",
+    "macaq_w4a4_grouped_linear_device", "grouped_device_workspace_bytes",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
@@ -39,7 +40,7 @@ EXPORTED_SYMBOLS = (
     "macaq_act_quant_plain", "macaq_mxfp4_linear", "macaq_mxfp4_gemm", "macaq_device_status",
     "macaq_grouped_workspace_bytes", "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc",
     "macaq_hessian_workspace_bytes", "macaq_calib_hessian", "macaq_flip_refine_workspace_bytes",
-    "macaq_flip_refine",
+    "macaq_flip_refine", "macaq_grouped_device_workspace_bytes", "macaq_w4a4_grouped_linear_device",
 )
 
 MACAQ_OK = 0
@@ -93,10 +94,13 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_flip_refine_workspace_bytes.argtypes = [i64, i64]
         lib.macaq_flip_refine_workspace_bytes.restype = sz
         lib.macaq_flip_refine.argtypes = [p, i64, i64, p, p, p, p, i64, p, p, sz, p]
+        lib.macaq_grouped_device_workspace_bytes.argtypes = [i64, i32, i64, i64]
+        lib.macaq_grouped_device_workspace_bytes.restype = sz
+        lib.macaq_w4a4_grouped_linear_device.argtypes = [p, i64, p, i32, i32, i64, p, p, p, i64, p, p, sz, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian",
-                     "macaq_flip_refine"):
+                     "macaq_flip_refine", "macaq_w4a4_grouped_linear_device"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -356,6 +360,43 @@ def macaq_w4a4_grouped_linear(x: torch.Tensor, counts, act_mult, Wq: torch.Tenso
     return y
 
 
+def grouped_device_workspace_bytes(T: int, E: int, N: int, K: int, device=None) -> int:
+    """Scratch bytes macaq_w4a4_grouped_linear_device needs for T routed rows over E experts."""
+    with _device(device):
+        return int(load_library().macaq_grouped_device_workspace_bytes(T, E, N, K))
+
+
+def macaq_w4a4_grouped_linear_device(x: torch.Tensor, counts: torch.Tensor, act_mult, Wq: torch.Tensor,
+                                     Ws: torch.Tensor, N: int, y=None, workspace=None, stream=None):
+    """Grouped (mixture-of-experts) linear with the per-expert token counts on the DEVICE (int32 or
+    int64 CUDA tensor [E], e.g. straight from a GPU router): no host copy, no synchronisation.  x
+    [T, K] bf16 grouped by expert, act_mult fp32 [E, K] (None: plain MXFP4), Wq [E, N, K/2], Ws the
+    experts' scale buffers concatenated.  Returns y bf16 [T, N]."""
+    T, K = x.shape
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    if counts.dtype not in (torch.int32, torch.int64):
+        raise ValueError("counts must be int32 or int64")
+    _need(counts, "counts", counts.dtype, device=dev)
+    E = counts.numel()
+    if act_mult is not None:
+        _need(act_mult, "act_mult", torch.float32, (E, K), device=dev)
+    _need(Wq, "Wq", torch.uint8, (E, N, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=E * scale_bytes(N, K), device=dev)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (T, N), device=dev)
+    need = grouped_device_workspace_bytes(T, E, N, K, dev)
+    if need == 0:
+        raise ValueError("shape not supported by the grouped linear (1 <= E <= 128, N % 128 == 0, T >= 1)")
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, min_numel=need, device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_w4a4_grouped_linear_device(
+            _ptr(x), T, _ptr(counts), counts.element_size(), E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+            _ptr(workspace), workspace.numel(), _stream(stream, dev)), "macaq_w4a4_grouped_linear_device")
+    return y
+
+
 NOALLOC_SCRATCH_BYTES = 32 << 20  # MACAQ_NOALLOC_SCRATCH_BYTES of include/macaq.h
 
 
@@ -423,5 +464,6 @@ def macaq_flip_refine(W: torch.Tensor, s: torch.Tensor, Hs: torch.Tensor, Wq: to
 
 
 def macaq_device_status(clear: bool = False) -> int:
-    """MACAQ_OK, or MACAQ_ETIMEOUT if a bounded device-side wait gave up (synchronises)."""
+    """MACAQ_OK, or the last device-side event: MACAQ_ETIMEOUT (a bounded wait gave up) or
+    MACAQ_ECOUNTS (device routing counts were corrected).  Synchronises."""
     return int(load_library().macaq_device_status(1 if clear else 0))

@@ -33,6 +33,8 @@ extern "C" const char* macaq_status_str(int status) {
         case MACAQ_EWORKSPACE: return "MACAQ_EWORKSPACE: workspace too small";
         case MACAQ_ETOOLARGE:
             return "MACAQ_ETOOLARGE: problem needs more scratch than the no-allocation entry point holds";
+        case MACAQ_ECOUNTS:
+            return "MACAQ_ECOUNTS: device routing counts were negative or ran past the rows of x (corrected)";
         default: return "MACAQ: unknown status";
     }
 }
@@ -56,5 +58,5 @@ extern "C" int macaq_device_status(int clear) {
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MACAQ_ECUDA;
     }
-    return v == 0 ? MACAQ_OK : MACAQ_ETIMEOUT;
+    return v;  // MACAQ_OK, or the code of the last event recorded (MACAQ_ETIMEOUT, MACAQ_ECOUNTS)
 }

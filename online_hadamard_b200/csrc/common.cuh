@@ -61,6 +61,23 @@ struct RowRuns {
     int run_start[kMaxGroups + 1];
 };
 
+// Where the grouped kernels find the expert table: passed by value (built on the host from host
+// counts) or in device memory (built by a kernel from device counts, so a router on the GPU needs
+// no device-to-host copy).
+struct HostGroups {
+    GroupTable gt;
+    RowRuns rr;
+};
+struct DeviceGroups {
+    const GroupTable* gt;
+    const RowRuns* rr;
+};
+__host__ __device__ __forceinline__ const GroupTable& group_table(const GroupTable& g) { return g; }
+__host__ __device__ __forceinline__ const GroupTable& group_table(const HostGroups& g) { return g.gt; }
+__host__ __device__ __forceinline__ const GroupTable& group_table(const DeviceGroups& g) { return *g.gt; }
+__host__ __device__ __forceinline__ const RowRuns& row_runs(const HostGroups& g) { return g.rr; }
+__host__ __device__ __forceinline__ const RowRuns& row_runs(const DeviceGroups& g) { return *g.rr; }
+
 // The expert whose range [starts[e], starts[e + 1]) holds v (0 <= v < starts[E]); empty ranges
 // are skipped.
 __host__ __device__ __forceinline__ int group_of(const int* starts, int groups, int v) {

@@ -51,6 +51,9 @@ int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq,
                            cudaStream_t stream);
 int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult, uint8_t* Aq, uint8_t* As,
                              const GroupTable& gt, cudaStream_t stream);
+int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
+                                    uint8_t* As, const DeviceGroups& dg, cudaStream_t stream);
+int64_t device_groups_rpg(int64_t T, int64_t K);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -104,6 +107,7 @@ struct GemmParams {
     int num_p_tiles, num_q_tiles, num_k_tiles, q_row_blocks;
     int raster_group;     // pair kernel: activation panels per group of the tile order (pair_tile)
     int dp_tiles;         // tiles scheduled data-parallel (blockIdx.x + i * gridDim.x)
+    const int* dp_tiles_dev;  // if set: the data-parallel tile count in device memory (device-built expert table)
     int64_t sk_units;     // K steps of the remaining tiles, split evenly over the first sk_count units
     int sk_count;         // scheduling units that take part in the split (<= the units launched)
     int64_t group_n;      // grouped linear: output features per expert (weights stacked [E][N][K])
@@ -190,12 +194,13 @@ struct Work {
 };
 
 struct WorkIter {
-    int dp_next, id, count;
+    int dp_next, id, count, dp_tiles;
     int64_t pos, hi;
 
     // `id` of `count` scheduling units: the CTA for the one-CTA kernel, the CTA pair for the
     // pair kernel (both CTAs of a pair walk the same items).
     __device__ __forceinline__ WorkIter(const GemmParams& p, int id_, int count_) : id(id_), count(count_) {
+        dp_tiles = p.dp_tiles_dev ? *p.dp_tiles_dev : p.dp_tiles;
         dp_next = id;
         pos = id < p.sk_count ? p.sk_units * id / p.sk_count : 0;
         hi = id < p.sk_count ? p.sk_units * (id + 1) / p.sk_count : 0;
@@ -203,7 +208,7 @@ struct WorkIter {
 
     __device__ __forceinline__ bool next(const GemmParams& p, Work& w) {
         const int KT = p.num_k_tiles;
-        if (dp_next < p.dp_tiles) {
+        if (dp_next < dp_tiles) {
             w.tile = dp_next;
             w.k0 = 0;
             w.k1 = KT;
@@ -216,7 +221,7 @@ struct WorkIter {
         const int64_t ts = pos / KT;
         const int64_t t0 = ts * KT;
         const int64_t end = hi < t0 + KT ? hi : t0 + KT;
-        w.tile = p.dp_tiles + static_cast<int>(ts);
+        w.tile = dp_tiles + static_cast<int>(ts);
         w.k0 = static_cast<int>(pos - t0);
         w.k1 = static_cast<int>(end - t0);
         if (w.k0 == 0 && w.k1 == KT) {
@@ -429,7 +434,7 @@ struct TileRef {
 };
 
 template <int BN, bool SWAP, bool GROUPED, class GT>
-__device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& gt, int tile) {
+__device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& groups, int tile) {
     TileRef t;
     if constexpr (!GROUPED) {
         const int pt = tile % prm.num_p_tiles, qt = tile / prm.num_p_tiles;
@@ -440,6 +445,7 @@ __device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& gt,
         t.p_end = prm.p_rows;
         t.q_end = prm.q_rows;
     } else {
+        const GroupTable& gt = group_table(groups);
         const int e = group_of(gt.tile_start, gt.groups, tile);
         const int local = tile - gt.tile_start[e];
         const int64_t rows = gt.rows[e], N = prm.group_n;
@@ -1170,11 +1176,11 @@ struct GemmScratch {
 };
 
 // Shared-memory attributes of one kernel instantiation, set once per device.
-template <int BN, int STAGES, bool SWAP, bool GROUPED>
+template <int BN, int STAGES, bool SWAP, bool GROUPED, class GT>
 static bool kernel_attributes() {
     static int cache[64] = {0};
     return cached_per_device(cache, [] {
-               auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP, GROUPED>;
+               auto kernel = mxf4_gemm_kernel<BN, STAGES, SWAP, GROUPED, GT>;
                const int smem = smem_bytes<BN, STAGES, SWAP>();
                cudaFuncAttributes fa;
                if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || !register_split_fits(fa)) {
@@ -1188,13 +1194,22 @@ static bool kernel_attributes() {
            }) == 1;
 }
 
-// GROUPED: `groups` maps the work tiles to experts (data-parallel schedule, no scratch); the
-// operands are the padded activation codes and the stacked weights, y is [tokens][N].
-template <int BN, int STAGES, bool SWAP, bool GROUPED = false>
+// Shape of a grouped launch: rows of y, the tile count (an upper bound when the expert table is in
+// device memory, whose own count `tiles_dev` the kernel reads), output features per expert.
+struct GroupedShape {
+    int64_t y_rows, tiles, group_n;
+    const int* tiles_dev;
+};
+
+// GT = GroupTable (host-built, by value) or DeviceGroups (device-built): `groups` maps the work tiles
+// to experts (data-parallel schedule, no scratch); the operands are the padded activation codes and
+// the stacked weights, y is [tokens][N].  GT = NoGroups: a plain GEMM.
+template <int BN, int STAGES, bool SWAP, class GT = NoGroups>
 static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream_t stream, bool pdl,
-                       const GroupTable* groups = nullptr, int64_t group_n = 0) {
+                       const GT& groups = GT{}, const GroupedShape* gs = nullptr) {
     using Cfg = TileCfg<BN>;
-    if (GROUPED && !kernel_attributes<BN, STAGES, SWAP, GROUPED>()) return MACAQ_ECUDA;
+    constexpr bool GROUPED = !std::is_same<GT, NoGroups>::value;
+    if (GROUPED && !kernel_attributes<BN, STAGES, SWAP, GROUPED, GT>()) return MACAQ_ECUDA;
     CUtensorMap mp, mq;
     if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, op.q_rows, op.K, BN))
         return MACAQ_ECUDA;
@@ -1217,15 +1232,15 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     if (ctas < 1) return MACAQ_ECUDA;
     CUtensorMap my;
     // y is [p_rows][q_rows], or for a grouped linear [tokens][group_n]
-    const int64_t y_rows = GROUPED ? groups->x_row[groups->groups - 1] + groups->rows[groups->groups - 1] : op.p_rows;
-    const int64_t y_cols = GROUPED ? group_n : op.q_rows;
+    const int64_t y_rows = GROUPED ? gs->y_rows : op.p_rows;
+    const int64_t y_cols = GROUPED ? gs->group_n : op.q_rows;
     prm.tma_store = (!SWAP && !op.y_fp32 && op.ldy % 8 == 0) ? 1 : 0;
     if (prm.tma_store && !make_out_map(&my, op.y, y_rows, y_cols, op.ldy)) return MACAQ_ECUDA;
     if (!prm.tma_store) my = mq;  // unused placeholder
-    const int64_t tiles = GROUPED ? groups->tile_start[groups->groups]
-                                  : static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
+    const int64_t tiles = GROUPED ? gs->tiles : static_cast<int64_t>(prm.num_p_tiles) * prm.num_q_tiles;
     if (tiles == 0) return MACAQ_OK;
-    prm.group_n = group_n;
+    prm.group_n = GROUPED ? gs->group_n : 0;
+    prm.dp_tiles_dev = GROUPED ? gs->tiles_dev : nullptr;
     const bool scratch = !GROUPED && ws.ptr != nullptr && ws.bytes >= streamk_bytes<BN>(ctas);
     const Schedule sch = plan_schedule(tiles, ctas, prm.num_k_tiles, scratch, streamk_cost_steps<BN>());
     const int64_t grid = sch.grid;
@@ -1252,7 +1267,8 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     if constexpr (GROUPED) {
-        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP, true>, mp, mq, my, prm, *groups) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP, true, GT>, mp, mq, my, prm, groups) !=
+            cudaSuccess)
             return MACAQ_ECUDA;
     } else {
         if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP>, mp, mq, my, prm, NoGroups{}) != cudaSuccess)
@@ -1485,6 +1501,72 @@ static int build_group_table(const int64_t* counts, int E, int64_t N, GroupTable
     return MACAQ_OK;
 }
 
+// The expert table from DEVICE counts (int32 or int64 [E]): the same quantities build_group_table
+// computes on the host, plus the quantiser's runs of `rpg` rows.  One thread; E <= 128.  Counts are
+// made safe before use -- a negative count becomes 0 and a count that would run past the T rows of x
+// is cut at T -- and either correction records MACAQ_ECOUNTS in the device status, so no kernel ever
+// indexes outside x, y or the workspace.  `swap`: every expert fits one swap-AB tile (T <= 128).
+__global__ void build_groups_kernel(const void* __restrict__ counts, int counts_bytes, int E, int64_t T, int64_t N,
+                                    int swap, int rpg, GroupTable* __restrict__ gt, RowRuns* __restrict__ rr) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    int bad = 0;
+    int64_t x = 0, a = 0, t = 0, runs = 0;
+    gt->groups = E;
+    for (int e = 0; e < E; ++e) {
+        int64_t c = counts_bytes == 4 ? static_cast<int64_t>(static_cast<const int32_t*>(counts)[e])
+                                      : static_cast<const int64_t*>(counts)[e];
+        if (c < 0) {
+            c = 0;
+            bad = 1;
+        }
+        if (c > T - x) {
+            c = T - x;
+            bad = 1;
+        }
+        gt->rows[e] = static_cast<int>(c);
+        gt->x_row[e] = static_cast<int>(x);
+        gt->a_row[e] = static_cast<int>(a);
+        gt->tile_start[e] = static_cast<int>(t);
+        rr->run_start[e] = static_cast<int>(runs);
+        x += c;
+        a += (c + 127) / 128 * 128;
+        if (c > 0) t += swap ? N / 128 : (c + 127) / 128 * ((N + 255) / 256);
+        runs += (c + rpg - 1) / rpg;
+    }
+    gt->a_row[E] = static_cast<int>(a);
+    gt->tile_start[E] = static_cast<int>(t);
+    rr->run_start[E] = static_cast<int>(runs);
+    rr->rpg = rpg;
+    if (bad) atomicExch(&g_device_status, MACAQ_ECOUNTS);
+}
+
+// Layout of the device-count grouped linear's workspace: the expert table, the quantiser's runs,
+// then the activation codes and scales for the most padded rows T tokens can need over E experts
+// (each non-empty expert pads to whole 128-row blocks: T + 127 min(E, T), rounded up to 128).
+struct DeviceGroupedWorkspace {
+    GroupTable* gt;
+    RowRuns* rr;
+    uint8_t *Aq, *As;
+    int64_t P;  // padded rows the codes can hold
+    size_t bytes;
+};
+
+static DeviceGroupedWorkspace device_grouped_layout(void* base, int64_t T, int E, int64_t K) {
+    DeviceGroupedWorkspace l;
+    const int64_t nz = E < T ? E : T;
+    l.P = (T + 127 * nz + 127) / 128 * 128;
+    const size_t off_rr = round256(sizeof(GroupTable));
+    const size_t off_aq = off_rr + round256(sizeof(RowRuns));
+    const size_t off_as = off_aq + round256(static_cast<size_t>(l.P * (K / 2)));
+    l.bytes = off_as + round256(static_cast<size_t>(scale_bytes(l.P, K)));
+    uint8_t* p = static_cast<uint8_t*>(base);
+    l.gt = reinterpret_cast<GroupTable*>(p);
+    l.rr = reinterpret_cast<RowRuns*>(p + off_rr);
+    l.Aq = p + off_aq;
+    l.As = p + off_as;
+    return l;
+}
+
 size_t grouped_activation_bytes(int64_t padded_rows, int64_t K) {
     return round256(static_cast<size_t>(padded_rows * (K / 2))) +
            round256(static_cast<size_t>(scale_bytes(padded_rows, K)));
@@ -1574,21 +1656,71 @@ extern "C" int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* count
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (int rc = launch_act_quant_grouped(x, K, act_mult, Aq, As, gt, st)) return rc;
     const GemmScratch none{nullptr, 0};
+    const GroupedShape gs{gt.x_row[E - 1] + gt.rows[E - 1], gt.tile_start[E], N, nullptr};
     if (mx <= 128) {  // decode-sized experts: weights on the MMA's 128-row side, tokens as N
         return with_config(mx, [&](auto bn, auto stages, auto sw) -> int {
             if constexpr (decltype(sw)::value) {
                 const GemmOperands op{Wq, Ws, Aq, As, E * N, P, K, y, N, 0};
-                return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, true>(op, none, st, true, &gt, N);
+                return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, GroupTable>(op, none, st, true,
+                                                                                                   gt, &gs);
             } else {
                 return MACAQ_EINVAL;  // not reached: up to 128 tokens always take a swap-AB configuration
             }
         });
     }
     const GemmOperands op{Aq, As, Wq, Ws, P, E * N, K, y, N, 0};
-    return launch_gemm<256, 4, false, true>(op, none, st, true, &gt, N);
+    return launch_gemm<256, 4, false, GroupTable>(op, none, st, true, gt, &gs);
 }
 
 #ifdef MACAQ_TEST_HOOKS
 // Fault injection (test build only): offset of the tag stream-K owners wait for.
 extern "C" void macaq_test_owner_tag_offset(int64_t offset) { macaq::g_test_owner_tag_offset.store(offset); }
 #endif
+
+extern "C" size_t macaq_grouped_device_workspace_bytes(int64_t T, int E, int64_t N, int64_t K) {
+    if (check_shape(T, K) || E < 1 || E > kMaxGroups || N < 128 || N % 128 != 0 || N > kMaxDim) return 0;
+    if (T + 127 * static_cast<int64_t>(E) + 128 > kMaxDim) return 0;
+    return device_grouped_layout(nullptr, T, E, K).bytes;
+}
+
+extern "C" int macaq_w4a4_grouped_linear_device(const uint16_t* x, int64_t T, const void* counts, int counts_bytes,
+                                                int E, int64_t K, const float* act_mult, const uint8_t* Wq,
+                                                const uint8_t* Ws, int64_t N, uint16_t* y, void* workspace,
+                                                size_t workspace_bytes, void* stream) {
+    if (!x || !counts || !Wq || !Ws || !y || !workspace) return MACAQ_EINVAL;
+    if (counts_bytes != 4 && counts_bytes != 8) return MACAQ_EINVAL;
+    if (int st = check_shape(T, K)) return st;
+    if (E < 1 || E > kMaxGroups) return MACAQ_ESHAPE;
+    if (N < 128 || N % 128 != 0 || N > kMaxDim || static_cast<int64_t>(E) * N > kMaxDim) return MACAQ_ESHAPE;
+    if (T + 127 * static_cast<int64_t>(E) + 128 > kMaxDim) return MACAQ_ESHAPE;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y) || !aligned16(workspace) ||
+        (act_mult && !aligned16(act_mult)) || (reinterpret_cast<uintptr_t>(counts) % counts_bytes) != 0)
+        return MACAQ_EALIGN;
+    const DeviceGroupedWorkspace l = device_grouped_layout(workspace, T, E, K);
+    if (workspace_bytes < l.bytes) return MACAQ_EWORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool swap = T <= 128;  // every expert then fits one swap-AB tile of the narrowest N holding T
+    const int64_t rpg = device_groups_rpg(T, K);
+    build_groups_kernel<<<1, 32, 0, st>>>(counts, counts_bytes, E, T, N, swap ? 1 : 0, static_cast<int>(rpg), l.gt,
+                                          l.rr);
+    if (int rc = launch_status()) return rc;
+    const DeviceGroups dg{l.gt, l.rr};
+    if (int rc = launch_act_quant_grouped_device(x, T, E, K, act_mult, l.Aq, l.As, dg, st)) return rc;
+    const GemmScratch none{nullptr, 0};
+    const int64_t nz = E < T ? E : T;
+    if (swap) {
+        const GroupedShape gs{T, nz * (N / 128), N, &l.gt->tile_start[E]};
+        return with_config(T, [&](auto bn, auto stages, auto sw) -> int {
+            if constexpr (decltype(sw)::value) {
+                const GemmOperands op{Wq, Ws, l.Aq, l.As, E * N, l.P, K, y, N, 0};
+                return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, DeviceGroups>(op, none, st, true,
+                                                                                                     dg, &gs);
+            } else {
+                return MACAQ_EINVAL;  // not reached: up to 128 tokens always take a swap-AB configuration
+            }
+        });
+    }
+    const GroupedShape gs{T, (T / 128 + nz + 1) * ((N + 255) / 256), N, &l.gt->tile_start[E]};
+    const GemmOperands op{l.Aq, l.As, Wq, Ws, l.P, E * N, K, y, N, 0};
+    return launch_gemm<256, 4, false, DeviceGroups>(op, none, st, true, dg, &gs);
+}

@@ -257,12 +257,14 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_kernel(
 // padded codes, quantised with the expert's own multipliers (act_mult + e K, transform mode).
 // The padding rows up to the next 128-row boundary are left as they are: they reach only rows
 // of the GEMM's output tile that are never stored.
-template <QuantMode MODE, bool AHEAD = false>
+template <QuantMode MODE, bool AHEAD = false, class SRC = HostGroups>
 __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
     const uint16_t* __restrict__ x, int64_t K, const float* __restrict__ act_mult, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, const __grid_constant__ GroupTable gt, const __grid_constant__ RowRuns rr) {
+    uint8_t* __restrict__ scales, const __grid_constant__ SRC src) {
     static_assert(MODE != QuantMode::kWeightFold, "activations only");
     griddep_launch_dependents();
+    const GroupTable& gt = group_table(src);
+    const RowRuns& rr = row_runs(src);
     const int64_t kbp = padded_blocks(K);
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
     const int64_t kb = item % kbp;
@@ -479,18 +481,43 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
         if (kbp * runs(mid) <= quant_thread_target()) hi = mid;
         else lo = mid + 1;
     }
-    RowRuns rr;
-    rr.rpg = lo;
-    rr.run_start[0] = 0;
-    for (int e = 0; e < gt.groups; ++e) rr.run_start[e + 1] = rr.run_start[e] + (gt.rows[e] + lo - 1) / lo;
-    const int64_t items = kbp * rr.run_start[gt.groups];
+    HostGroups hg;
+    hg.gt = gt;
+    hg.rr.rpg = lo;
+    hg.rr.run_start[0] = 0;
+    for (int e = 0; e < gt.groups; ++e) hg.rr.run_start[e + 1] = hg.rr.run_start[e] + (gt.rows[e] + lo - 1) / lo;
+    const int64_t items = kbp * hg.rr.run_start[gt.groups];
     const unsigned blocks = static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
     if (act_mult) {
         const auto kernel = tokens * K >= kAheadMinElems ? mx_quant_grouped_kernel<QuantMode::kActTransform, true>
                                                          : mx_quant_grouped_kernel<QuantMode::kActTransform, false>;
-        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, gt, rr);
+        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, hg);
     } else {
-        mx_quant_grouped_kernel<QuantMode::kPlain><<<blocks, kQuantThreads, 0, stream>>>(x, K, nullptr, Aq, As, gt, rr);
+        mx_quant_grouped_kernel<QuantMode::kPlain><<<blocks, kQuantThreads, 0, stream>>>(x, K, nullptr, Aq, As, hg);
+    }
+    return launch_status();
+}
+
+// Rows per run of the grouped quantiser when only the total T of routed rows and the expert count
+// are known on the host (device counts): runs of quant_rows_per_thread(T) rows, and a grid for the
+// most runs any split of T rows over E experts can need (T / rpg + E); threads past the real runs
+// return at once.
+int64_t device_groups_rpg(int64_t T, int64_t K) { return quant_rows_per_thread(T, K); }
+int64_t device_groups_max_runs(int64_t T, int E, int64_t rpg) { return T / rpg + E; }
+
+int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
+                                    uint8_t* As, const DeviceGroups& dg, cudaStream_t stream) {
+    const int64_t rpg = device_groups_rpg(T, K);
+    const int64_t items = padded_blocks(K) * device_groups_max_runs(T, E, rpg);
+    const unsigned blocks = static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
+    if (act_mult) {
+        const auto kernel = T * K >= kAheadMinElems
+                                ? mx_quant_grouped_kernel<QuantMode::kActTransform, true, DeviceGroups>
+                                : mx_quant_grouped_kernel<QuantMode::kActTransform, false, DeviceGroups>;
+        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, dg);
+    } else {
+        mx_quant_grouped_kernel<QuantMode::kPlain, false, DeviceGroups><<<blocks, kQuantThreads, 0, stream>>>(
+            x, K, nullptr, Aq, As, dg);
     }
     return launch_status();
 }

@@ -91,3 +91,44 @@ def test_grouped_without_tokens_leaves_y_alone(mq):
     y = mq.macaq_w4a4_grouped_linear(x, [0, 0, 0], am, Wq, Ws, N)
     torch.cuda.synchronize()
     assert y.shape == (0, N)
+
+
+@pytest.mark.parametrize("name,counts,N,K", CASES, ids=[c[0] for c in CASES])
+@pytest.mark.parametrize("dtype", [torch.int32, torch.int64], ids=["i32", "i64"])
+def test_device_counts_match_host_counts(mq, name, counts, N, K, dtype):
+    """The counts on the device (a GPU router's output): y matches the host-count call within the
+    GEMM tolerance (the kernel choice may differ: the host call picks it from the largest expert, the
+    device call from the total), and both match the oracle per expert via the test above."""
+    E, T = len(counts), sum(counts)
+    Wq, Ws, am = _experts(mq, E, N, K, seed=E * 31 + N + K)
+    g = torch.Generator().manual_seed(T + K)
+    x = (torch.randn(T, K, generator=g) * 2).to(torch.bfloat16).cuda()
+    host = mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N)
+    ws = torch.full((mq.grouped_device_workspace_bytes(T, E, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
+    dev = mq.macaq_w4a4_grouped_linear_device(x, torch.tensor(counts, dtype=dtype, device="cuda"), am, Wq, Ws, N,
+                                              workspace=ws)
+    dev2 = mq.macaq_w4a4_grouped_linear_device(x, torch.tensor(counts, dtype=dtype, device="cuda"), None, Wq, Ws, N)
+    plain = mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status() == 0
+    assert bool(torch.isfinite(dev.float()).all())
+    assert gu.rel_fro(gu.to_np(dev.float()), gu.to_np(host.float())) <= TOL
+    assert gu.rel_fro(gu.to_np(dev2.float()), gu.to_np(plain.float())) <= TOL
+
+
+def test_device_counts_out_of_range_are_corrected_and_reported(mq):
+    """Negative counts or counts past the rows of x are corrected on the device (no access outside x
+    or y) and reported as MACAQ_ECOUNTS; the rows they do cover are computed as usual."""
+    N, K = 256, 512
+    Wq, Ws, am = _experts(mq, 3, N, K, seed=9)
+    x = (torch.randn(40, K) * 2).to(torch.bfloat16).cuda()
+    ref = mq.macaq_w4a4_grouped_linear(x[:30], [10, 0, 20], am, Wq, Ws, N)
+    y = torch.zeros(40, N, dtype=torch.bfloat16, device="cuda")
+    mq.macaq_w4a4_grouped_linear_device(x, torch.tensor([10, -5, 1000], dtype=torch.int32, device="cuda"), am, Wq, Ws,
+                                        N, y=y)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status(clear=True) == -8  # MACAQ_ECOUNTS
+    assert mq.macaq_device_status() == 0
+    # expert 2's count is cut at the 30 rows that remain after expert 0: rows 10..39
+    assert gu.rel_fro(gu.to_np(y[:10].float()), gu.to_np(ref[:10].float())) <= TOL
+    assert bool(torch.isfinite(y.float()).all())
