@@ -654,6 +654,10 @@ def summary(out):
         if isinstance(v, dict):
             sm["moe_" + k] = {"us": r(v["ms"] * 1e3), "roof": r(v["linear_roofline_frac"]),
                               "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2)}
+    fl = sec.get("flip_refinement")
+    if fl:
+        sm["flip_llama_up"] = {"ms": r(fl["hessian_ms"] + fl["refine_ms"]),
+                               "err_rtn": r(fl["held_out_rel_err_rtn"]), "err_refined": r(fl["held_out_rel_err_refined"])}
     par = out.get("parity")
     if par:
         sm["parity_cfg4"] = {"ok": par["ok"], "exempt": par["activations"]["exempt"] + par["weights"]["exempt"],
@@ -758,9 +762,13 @@ def moe_sweep(mq, device, peaks, token_counts=(16, 4096), steps=10, warmup=3):
                                                layer=E * li + E), rows, device)
             y = torch.empty(rows, N, dtype=torch.bfloat16, device=device)
             ws = torch.empty(max(mq.grouped_workspace_bytes(counts, N, K), 1), dtype=torch.uint8, device=device)
+            counts_dev = torch.tensor(counts, dtype=torch.int32, device=device)
+            ws_dev = torch.empty(mq.grouped_device_workspace_bytes(rows, E, N, K), dtype=torch.uint8, device=device)
             ab = time_ab({"w4a4": lambda i: mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N, y=y, workspace=ws),
                           "plain": lambda i: mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N, y=y,
-                                                                          workspace=ws)},
+                                                                          workspace=ws),
+                          "device": lambda i: mq.macaq_w4a4_grouped_linear_device(x, counts_dev, am, Wq, Ws, N,
+                                                                                  capacity=T, y=y, workspace=ws_dev)},
                          steps, warmup, device)
             ms, ms_plain = ab["w4a4"], ab["plain"]
             active = sum(1 for c in counts if c)
@@ -768,19 +776,51 @@ def moe_sweep(mq, device, peaks, token_counts=(16, 4096), steps=10, warmup=3):
             nbytes = active * N * K * (0.5 + 1 / 32) + 2.0 * rows * (K + N) + 4.0 * K * active
             t_roof = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
             res[f"{name}_T{T}"] = {"routed_rows": rows, "active_experts": active, "max_rows": max(counts),
-                                    "ms": ms, "plain_mxfp4_ms": ms_plain,
+                                    "ms": ms, "plain_mxfp4_ms": ms_plain, "device_counts_ms": ab["device"],
                                     "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
                                     "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
                                     "linear_roofline_frac": t_roof / (ms * 1e-3)}
-            del x, y, ws
+            del x, y, ws, ws_dev, counts_dev
         del Wq, Ws, am
         torch.cuda.empty_cache()
     return res
 
 
+def flip_leg(mq, device, wl=wls.LLAMA_UP, calib_tokens=128, max_moves=64, held_out=256):
+    """Flip-Refinement (offline) of one layer: the Hessian of a calibration batch and the refinement of
+    its round-to-nearest codes, timed with CUDA events; moves per row; and what it buys -- the W4A4
+    linear's relative output error against the exact x W^T on held-out tokens (same distribution),
+    round-to-nearest against refined codes."""
+    W = wls.make_w(wl).to(device)
+    s = wls.make_s(wl, W.cpu()).to(device)
+    xcal = torch.cat([wls.make_xcal(wl), wls._draw_x(wl, calib_tokens - wls.CALIB_TOKENS, 7).to(torch.bfloat16)])
+    xcal = xcal.to(device)
+    Wq, Ws, am = mq.macaq_fold_weights(W, s)
+    rtn = Wq.clone()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize(device)
+    e[0].record()
+    Hs = mq.macaq_calib_hessian(xcal, am)
+    e[1].record()
+    moves = mq.macaq_flip_refine(W, s, Hs, Wq, Ws, max_moves)
+    e[2].record()
+    torch.cuda.synchronize(device)
+    xh = wls._draw_x(wl, held_out, 11).to(torch.bfloat16).to(device)
+    exact = xh.float() @ W.t()
+    rel = lambda y: float((y.float() - exact).norm() / exact.norm())
+    out = {"workload": wl.name, "calibration_tokens": calib_tokens, "max_moves_per_row": max_moves,
+           "hessian_ms": e[0].elapsed_time(e[1]), "refine_ms": e[1].elapsed_time(e[2]),
+           "moves_per_row": float(moves.float().mean()), "code_bytes_changed": float((Wq != rtn).float().mean()),
+           "held_out_rel_err_rtn": rel(mq.macaq_w4a4_linear(xh, am, rtn, Ws, wl.N)),
+           "held_out_rel_err_refined": rel(mq.macaq_w4a4_linear(xh, am, Wq, Ws, wl.N))}
+    del W, Hs, Wq, rtn, Ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def secondary(mq, device, peaks, args):
-    """The Llama-3-8B up projection (tensor-bound prefill) and decode (HBM-bound)."""
-    res = {}
+    """The Llama-3-8B up projection (tensor-bound prefill), decode (HBM-bound) and Flip-Refinement."""
+    res = {"flip_refinement": flip_leg(mq, device)}
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     wl = wls.LLAMA_UP
     layer = Layer(mq, wl, device)

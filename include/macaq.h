@@ -68,7 +68,7 @@ typedef enum {
     MACAQ_ETIMEOUT = -5,   /* a bounded device-side wait gave up (see macaq_device_status) */
     MACAQ_EWORKSPACE = -6, /* workspace smaller than the call needs */
     MACAQ_ETOOLARGE = -7,  /* problem needs more than the no-allocation scratch (below) */
-    MACAQ_ECOUNTS = -8     /* device routing counts were corrected (see macaq_w4a4_grouped_linear_device) */
+    MACAQ_ECOUNTS = -8     /* device routing counts were corrected or capped (macaq_w4a4_grouped_linear_device) */
 } macaq_status;
 
 /* Human-readable name of a status code (static storage). */
@@ -210,24 +210,29 @@ int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* counts, int E, i
  * macaq_w4a4_grouped_linear_device -- macaq_w4a4_grouped_linear with the per-expert token counts in
  * DEVICE memory, as a router on the GPU produces them: nothing is copied to the host and the call
  * never synchronises.  A first kernel builds the expert table on the device, then the grouped
- * quantiser and GEMM run from it; grids and the workspace are sized on the host from T and E.
+ * quantiser and GEMM run from it; grids and the workspace are sized on the host from T, E and the
+ * capacity.
  *   x         in   bf16 [T][K], the tokens grouped by expert (T, the routed rows, known on the host)
  *   counts    in   DEVICE int32 (counts_bytes = 4) or int64 (8) [E], 1 <= E <= 128
+ *   capacity  in   the most rows any expert may have (an expert capacity, known on the host: e.g. the
+ *                  token count for top-k routing to distinct experts); <= 0 or > T means T.  It
+ *                  picks the kernels: up to 128, the weights take the MMA's 128-row side (swap-AB,
+ *                  N of the narrowest tile holding the capacity); above, 128-token x 256-feature tiles
  *   act_mult, Wq, Ws, N, y   as for macaq_w4a4_grouped_linear
  *   workspace in   at least macaq_grouped_device_workspace_bytes(T, E, N, K) bytes (the table and
  *                  activation codes for the most padded rows T tokens can need: T + 127 min(E, T))
- * Counts are expected to be >= 0 and to sum to T.  A negative count is taken as 0 and a count that
- * would run past row T is cut there; either correction sets MACAQ_ECOUNTS in macaq_device_status.
- * Rows of y past the counts' sum are not written.  With T <= 128 the weights take the MMA's 128-row
- * side (swap-AB, N of the narrowest tile holding T); above, 128-token x 256-feature tiles.  Results
- * match macaq_w4a4_grouped_linear within the GEMM tolerance (its kernel choice follows the largest
- * expert, this one T), activation codes bit for bit.
+ * Counts are expected to be >= 0, at most the capacity, and to sum to T.  A negative count is taken
+ * as 0, a count that would run past row T is cut there, and an expert's rows beyond the capacity are
+ * not computed (x keeps its layout); each of these sets MACAQ_ECOUNTS in macaq_device_status.  Rows
+ * of y that are not computed are not written.  Results match macaq_w4a4_grouped_linear within the
+ * GEMM tolerance (its kernel choice follows the largest expert, this one the capacity), activation
+ * codes bit for bit.
  */
 size_t macaq_grouped_device_workspace_bytes(int64_t T, int E, int64_t N, int64_t K);
 int macaq_w4a4_grouped_linear_device(const uint16_t* x, int64_t T, const void* counts, int counts_bytes, int E,
-                                     int64_t K, const float* act_mult, const uint8_t* Wq, const uint8_t* Ws,
-                                     int64_t N, uint16_t* y, void* workspace, size_t workspace_bytes,
-                                     void* stream);
+                                     int64_t capacity, int64_t K, const float* act_mult, const uint8_t* Wq,
+                                     const uint8_t* Ws, int64_t N, uint16_t* y, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * macaq_w4a4_linear_noalloc -- macaq_w4a4_linear for callers that cannot allocate device

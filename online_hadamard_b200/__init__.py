@@ -96,7 +96,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_flip_refine.argtypes = [p, i64, i64, p, p, p, p, i64, p, p, sz, p]
         lib.macaq_grouped_device_workspace_bytes.argtypes = [i64, i32, i64, i64]
         lib.macaq_grouped_device_workspace_bytes.restype = sz
-        lib.macaq_w4a4_grouped_linear_device.argtypes = [p, i64, p, i32, i32, i64, p, p, p, i64, p, p, sz, p]
+        lib.macaq_w4a4_grouped_linear_device.argtypes = [p, i64, p, i32, i32, i64, i64, p, p, p, i64, p, p, sz, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian",
@@ -367,11 +367,13 @@ def grouped_device_workspace_bytes(T: int, E: int, N: int, K: int, device=None) 
 
 
 def macaq_w4a4_grouped_linear_device(x: torch.Tensor, counts: torch.Tensor, act_mult, Wq: torch.Tensor,
-                                     Ws: torch.Tensor, N: int, y=None, workspace=None, stream=None):
+                                     Ws: torch.Tensor, N: int, capacity: int = 0, y=None, workspace=None, stream=None):
     """Grouped (mixture-of-experts) linear with the per-expert token counts on the DEVICE (int32 or
     int64 CUDA tensor [E], e.g. straight from a GPU router): no host copy, no synchronisation.  x
     [T, K] bf16 grouped by expert, act_mult fp32 [E, K] (None: plain MXFP4), Wq [E, N, K/2], Ws the
-    experts' scale buffers concatenated.  Returns y bf16 [T, N]."""
+    experts' scale buffers concatenated; capacity = the most rows any expert may have (0: T), which
+    picks the kernels; rows past it are not computed (reported as MACAQ_ECOUNTS).  Returns y bf16
+    [T, N]."""
     T, K = x.shape
     _need(x, "x", torch.bfloat16)
     dev = x.device
@@ -392,7 +394,8 @@ def macaq_w4a4_grouped_linear_device(x: torch.Tensor, counts: torch.Tensor, act_
     _need(workspace, "workspace", torch.uint8, min_numel=need, device=dev)
     with torch.cuda.device(dev):
         _check(load_library().macaq_w4a4_grouped_linear_device(
-            _ptr(x), T, _ptr(counts), counts.element_size(), E, K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N, _ptr(y),
+            _ptr(x), T, _ptr(counts), counts.element_size(), E, int(capacity), K, _ptr(act_mult), _ptr(Wq), _ptr(Ws), N,
+            _ptr(y),
             _ptr(workspace), workspace.numel(), _stream(stream, dev)), "macaq_w4a4_grouped_linear_device")
     return y
 

@@ -53,7 +53,7 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
                              const GroupTable& gt, cudaStream_t stream);
 int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
                                     uint8_t* As, const DeviceGroups& dg, cudaStream_t stream);
-int64_t device_groups_rpg(int64_t T, int64_t K);
+int64_t device_groups_rpg(int64_t T, int E, int64_t K);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -470,6 +470,17 @@ __device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& gro
     return t;
 }
 
+// The expert table tile_ref reads: the kernel parameter (host-built table, or no groups), or the
+// shared-memory copy of a device-built table, so a tile's expert lookup (a binary search) reads
+// shared memory instead of a chain of dependent global loads.
+template <class GT>
+__device__ __forceinline__ const auto& tile_table(const GT& gt, const int* s_table) {
+    if constexpr (std::is_same<GT, DeviceGroups>::value)
+        return *reinterpret_cast<const GroupTable*>(s_table);
+    else
+        return gt;
+}
+
 // GROUPED: a grouped (mixture-of-experts) linear; `gt` maps work tiles to experts.
 template <int BN, int STAGES, bool SWAP, bool GROUPED = false,
           class GT = typename std::conditional<GROUPED, GroupTable, NoGroups>::type>
@@ -490,6 +501,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // A device-built expert table is copied to shared memory once (visible after the barrier below;
+    // it was written by a kernel that completed before the quantiser this GEMM follows had started).
+    constexpr bool kDevTable = std::is_same<GT, DeviceGroups>::value;
+    __shared__ __align__(16) int s_table[kDevTable ? sizeof(GroupTable) / 4 : 1];
+    if constexpr (kDevTable) {
+        const int* src = reinterpret_cast<const int*>(gt.gt);
+        for (int i = threadIdx.x; i < static_cast<int>(sizeof(GroupTable) / 4); i += blockDim.x) s_table[i] = src[i];
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -526,7 +545,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             WorkIter it(prm, blockIdx.x, gridDim.x);
             Work w;
             while (!abort && it.next(prm, w)) {
-                const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, gt, w.tile);
+                const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, tile_table(gt, s_table), w.tile);
                 const uint8_t* sfp = prm.sf_p + (t.p_row / 128) * (prm.kbp / 4) * 512;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
@@ -651,7 +670,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         WorkIter it(prm, blockIdx.x, gridDim.x);
         Work w;
         while (!abort && it.next(prm, w)) {
-            const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, gt, w.tile);
+            const TileRef t = tile_ref<BN, SWAP, GROUPED>(prm, tile_table(gt, s_table), w.tile);
             // Narrow tiles (decode): the owner of a split tile adds its contributors' partial
             // sums while its own MMAs still run.  The contributors did their part of the tile
             // first in their ranges; the owner reaches the tile's first K steps last in its own.
@@ -1502,42 +1521,94 @@ static int build_group_table(const int64_t* counts, int E, int64_t N, GroupTable
 }
 
 // The expert table from DEVICE counts (int32 or int64 [E]): the same quantities build_group_table
-// computes on the host, plus the quantiser's runs of `rpg` rows.  One thread; E <= 128.  Counts are
-// made safe before use -- a negative count becomes 0 and a count that would run past the T rows of x
-// is cut at T -- and either correction records MACAQ_ECOUNTS in the device status, so no kernel ever
-// indexes outside x, y or the workspace.  `swap`: every expert fits one swap-AB tile (T <= 128).
-__global__ void build_groups_kernel(const void* __restrict__ counts, int counts_bytes, int E, int64_t T, int64_t N,
-                                    int swap, int rpg, GroupTable* __restrict__ gt, RowRuns* __restrict__ rr) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    int bad = 0;
-    int64_t x = 0, a = 0, t = 0, runs = 0;
-    gt->groups = E;
-    for (int e = 0; e < E; ++e) {
-        int64_t c = counts_bytes == 4 ? static_cast<int64_t>(static_cast<const int32_t*>(counts)[e])
-                                      : static_cast<const int64_t*>(counts)[e];
-        if (c < 0) {
-            c = 0;
-            bad = 1;
-        }
-        if (c > T - x) {
-            c = T - x;
-            bad = 1;
-        }
-        gt->rows[e] = static_cast<int>(c);
-        gt->x_row[e] = static_cast<int>(x);
-        gt->a_row[e] = static_cast<int>(a);
-        gt->tile_start[e] = static_cast<int>(t);
-        rr->run_start[e] = static_cast<int>(runs);
-        x += c;
-        a += (c + 127) / 128 * 128;
-        if (c > 0) t += swap ? N / 128 : (c + 127) / 128 * ((N + 255) / 256);
-        runs += (c + rpg - 1) / rpg;
+// computes on the host, plus the quantiser's runs of `rpg` rows.  One CTA of 128 threads, one
+// expert each (E <= 128): the counts load in parallel, four running sums (x rows, padded rows,
+// tiles, runs) come from one block-wide exclusive scan, and every entry is stored in parallel.
+// Counts are made safe before use -- a negative count becomes 0 and a count that would run past
+// the T rows of x is cut at T -- and an expert's rows beyond `capacity` are not computed (x keeps
+// its layout); each correction records MACAQ_ECOUNTS in the device status, so no kernel ever indexes
+// outside x, y or the workspace.  `swap`: every expert fits one swap-AB tile (capacity <= 128).
+constexpr int kGroupThreads = kMaxGroups;
+
+__device__ __forceinline__ longlong4 add4(longlong4 a, longlong4 b) {
+    return make_longlong4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__global__ void __launch_bounds__(kGroupThreads) build_groups_kernel(
+    const void* __restrict__ counts, int counts_bytes, int E, int64_t T, int64_t capacity, int64_t N, int swap, int rpg,
+    GroupTable* __restrict__ gt, RowRuns* __restrict__ rr) {
+    __shared__ longlong4 warp_sum[kGroupThreads / 32];
+    __shared__ int64_t clamp_x[kGroupThreads];
+    __shared__ int bad;
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    if (e == 0) bad = 0;
+    __syncthreads();
+    int64_t c = 0;
+    if (e < E)
+        c = counts_bytes == 4 ? static_cast<int64_t>(static_cast<const int32_t*>(counts)[e])
+                              : static_cast<const int64_t*>(counts)[e];
+    if (c < 0) {
+        c = 0;
+        bad = 1;
     }
-    gt->a_row[E] = static_cast<int>(a);
-    gt->tile_start[E] = static_cast<int>(t);
-    rr->run_start[E] = static_cast<int>(runs);
-    rr->rpg = rpg;
-    if (bad) atomicExch(&g_device_status, MACAQ_ECOUNTS);
+    // 1. where expert e's rows start in x: exclusive scan of the counts, then the cut at T
+    int64_t incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int64_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sum[warp].x = incl;
+    __syncthreads();
+    int64_t before = incl - c;
+    for (int w = 0; w < warp; ++w) before += warp_sum[w].x;
+    const int64_t x0 = before < T ? before : T;
+    if (c > T - x0) {
+        c = T - x0;
+        bad = 1;
+    }
+    int64_t rows = c;
+    if (rows > capacity) {
+        rows = capacity;
+        bad = 1;
+    }
+    clamp_x[e] = x0;
+    __syncthreads();
+    // 2. padded rows, tiles and runs of the rows computed: one more scan
+    longlong4 v = make_longlong4((rows + 127) / 128 * 128,
+                                 rows > 0 ? (swap ? N / 128 : (rows + 127) / 128 * ((N + 255) / 256)) : 0,
+                                 (rows + rpg - 1) / rpg, 0);
+    longlong4 inc4 = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        longlong4 o;
+        o.x = __shfl_up_sync(0xFFFFFFFFu, inc4.x, off);
+        o.y = __shfl_up_sync(0xFFFFFFFFu, inc4.y, off);
+        o.z = __shfl_up_sync(0xFFFFFFFFu, inc4.z, off);
+        o.w = 0;
+        if (lane >= off) inc4 = add4(inc4, o);
+    }
+    __syncthreads();
+    if (lane == 31) warp_sum[warp] = inc4;
+    __syncthreads();
+    longlong4 pre = make_longlong4(inc4.x - v.x, inc4.y - v.y, inc4.z - v.z, 0);
+    for (int w = 0; w < warp; ++w) pre = add4(pre, warp_sum[w]);
+    if (e < E) {
+        gt->rows[e] = static_cast<int>(rows);
+        gt->x_row[e] = static_cast<int>(clamp_x[e]);
+        gt->a_row[e] = static_cast<int>(pre.x);
+        gt->tile_start[e] = static_cast<int>(pre.y);
+        rr->run_start[e] = static_cast<int>(pre.z);
+    }
+    if (e == E - 1) {
+        gt->groups = E;
+        gt->a_row[E] = static_cast<int>(pre.x + v.x);
+        gt->tile_start[E] = static_cast<int>(pre.y + v.y);
+        rr->run_start[E] = static_cast<int>(pre.z + v.z);
+        rr->rpg = rpg;
+    }
+    __syncthreads();
+    if (e == 0 && bad) atomicExch(&g_device_status, MACAQ_ECOUNTS);
 }
 
 // Layout of the device-count grouped linear's workspace: the expert table, the quantiser's runs,
@@ -1684,9 +1755,9 @@ extern "C" size_t macaq_grouped_device_workspace_bytes(int64_t T, int E, int64_t
 }
 
 extern "C" int macaq_w4a4_grouped_linear_device(const uint16_t* x, int64_t T, const void* counts, int counts_bytes,
-                                                int E, int64_t K, const float* act_mult, const uint8_t* Wq,
-                                                const uint8_t* Ws, int64_t N, uint16_t* y, void* workspace,
-                                                size_t workspace_bytes, void* stream) {
+                                                int E, int64_t capacity, int64_t K, const float* act_mult,
+                                                const uint8_t* Wq, const uint8_t* Ws, int64_t N, uint16_t* y,
+                                                void* workspace, size_t workspace_bytes, void* stream) {
     if (!x || !counts || !Wq || !Ws || !y || !workspace) return MACAQ_EINVAL;
     if (counts_bytes != 4 && counts_bytes != 8) return MACAQ_EINVAL;
     if (int st = check_shape(T, K)) return st;
@@ -1699,10 +1770,11 @@ extern "C" int macaq_w4a4_grouped_linear_device(const uint16_t* x, int64_t T, co
     const DeviceGroupedWorkspace l = device_grouped_layout(workspace, T, E, K);
     if (workspace_bytes < l.bytes) return MACAQ_EWORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool swap = T <= 128;  // every expert then fits one swap-AB tile of the narrowest N holding T
-    const int64_t rpg = device_groups_rpg(T, K);
-    build_groups_kernel<<<1, 32, 0, st>>>(counts, counts_bytes, E, T, N, swap ? 1 : 0, static_cast<int>(rpg), l.gt,
-                                          l.rr);
+    const int64_t cap = capacity < 1 || capacity > T ? T : capacity;  // rows per expert at most
+    const bool swap = cap <= 128;  // every expert then fits one swap-AB tile of the narrowest N holding cap
+    const int64_t rpg = device_groups_rpg(T, E, K);
+    build_groups_kernel<<<1, kGroupThreads, 0, st>>>(counts, counts_bytes, E, T, cap, N, swap ? 1 : 0,
+                                                     static_cast<int>(rpg), l.gt, l.rr);
     if (int rc = launch_status()) return rc;
     const DeviceGroups dg{l.gt, l.rr};
     if (int rc = launch_act_quant_grouped_device(x, T, E, K, act_mult, l.Aq, l.As, dg, st)) return rc;
@@ -1710,7 +1782,7 @@ extern "C" int macaq_w4a4_grouped_linear_device(const uint16_t* x, int64_t T, co
     const int64_t nz = E < T ? E : T;
     if (swap) {
         const GroupedShape gs{T, nz * (N / 128), N, &l.gt->tile_start[E]};
-        return with_config(T, [&](auto bn, auto stages, auto sw) -> int {
+        return with_config(cap, [&](auto bn, auto stages, auto sw) -> int {
             if constexpr (decltype(sw)::value) {
                 const GemmOperands op{Wq, Ws, l.Aq, l.As, E * N, l.P, K, y, N, 0};
                 return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, DeviceGroups>(op, none, st, true,

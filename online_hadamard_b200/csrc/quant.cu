@@ -263,8 +263,21 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
     uint8_t* __restrict__ scales, const __grid_constant__ SRC src) {
     static_assert(MODE != QuantMode::kWeightFold, "activations only");
     griddep_launch_dependents();
-    const GroupTable& gt = group_table(src);
-    const RowRuns& rr = row_runs(src);
+    // A device-built table is copied to shared memory first: each thread's expert lookup is a binary
+    // search, which would otherwise be a chain of dependent global loads.
+    constexpr bool kDevTable = std::is_same<SRC, DeviceGroups>::value;
+    constexpr int kTableWords = (sizeof(GroupTable) + sizeof(RowRuns)) / 4;
+    __shared__ __align__(16) int s_table[kDevTable ? kTableWords : 1];
+    if constexpr (kDevTable) {
+        const int* g = reinterpret_cast<const int*>(&group_table(src));
+        const int* r = reinterpret_cast<const int*>(&row_runs(src));
+        for (int i = threadIdx.x; i < kTableWords; i += blockDim.x)
+            s_table[i] = i < static_cast<int>(sizeof(GroupTable) / 4) ? g[i] : r[i - sizeof(GroupTable) / 4];
+        __syncthreads();
+    }
+    const GroupTable& gt = kDevTable ? *reinterpret_cast<const GroupTable*>(s_table) : group_table(src);
+    const RowRuns& rr = kDevTable ? *reinterpret_cast<const RowRuns*>(s_table + sizeof(GroupTable) / 4)
+                                  : row_runs(src);
     const int64_t kbp = padded_blocks(K);
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
     const int64_t kb = item % kbp;
@@ -499,15 +512,24 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
 }
 
 // Rows per run of the grouped quantiser when only the total T of routed rows and the expert count
-// are known on the host (device counts): runs of quant_rows_per_thread(T) rows, and a grid for the
-// most runs any split of T rows over E experts can need (T / rpg + E); threads past the real runs
-// return at once.
-int64_t device_groups_rpg(int64_t T, int64_t K) { return quant_rows_per_thread(T, K); }
+// are known on the host (device counts): the grid covers the most runs any split of T rows over E
+// experts can need, T / rpg + E, and threads past the real runs return at once.  The runs are made
+// long enough for that bound to fit one resident wave (as the host-count launch does for its actual
+// runs): a second wave would run nearly as long as the first.
+int64_t device_groups_rpg(int64_t T, int E, int64_t K) {
+    int64_t rpg = quant_rows_per_thread(T, K);
+    const int64_t wave_runs = quant_thread_target() / padded_blocks(K) - E;
+    if (wave_runs >= 1) {
+        const int64_t need = (T + wave_runs - 1) / wave_runs;
+        if (need > rpg) rpg = need;
+    }
+    return rpg;
+}
 int64_t device_groups_max_runs(int64_t T, int E, int64_t rpg) { return T / rpg + E; }
 
 int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
                                     uint8_t* As, const DeviceGroups& dg, cudaStream_t stream) {
-    const int64_t rpg = device_groups_rpg(T, K);
+    const int64_t rpg = device_groups_rpg(T, E, K);
     const int64_t items = padded_blocks(K) * device_groups_max_runs(T, E, rpg);
     const unsigned blocks = static_cast<unsigned>((items + kQuantThreads - 1) / kQuantThreads);
     if (act_mult) {

@@ -76,7 +76,9 @@ def test_summary_and_mx_diff_on_fake_results():
     lr = {"frac": 0.6}
     leg = {"roofline": {"frac": 0.7}, "overhead": {"vs_plain_mxfp4_pct": 3.0, "vs_gemm_only_pct": 9.0}}
     out = {"value": 4000.0, "linear_roofline": lr, **leg,
-           "secondary": {"llama3_8b_up_prefill": {"tflops": 4000.0, "linear_roofline": lr, **leg},
+           "secondary": {"flip_refinement": {"hessian_ms": 1.0, "refine_ms": 80.0, "held_out_rel_err_rtn": 0.062,
+                                             "held_out_rel_err_refined": 0.056},
+                         "llama3_8b_up_prefill": {"tflops": 4000.0, "linear_roofline": lr, **leg},
                          "qwen3_32b_up_decode_M1": {"gbs": 3600.0, "linear_roofline": lr, "vs_plain_mxfp4_pct": 2.0},
                          "qwen3_32b_stack": {"layers": 64, "M1": {"w4a4_ms": 6.5, "linear_roofline_frac": 0.4,
                                                                   "vs_plain_mxfp4_pct": 3.0}},
@@ -84,7 +86,8 @@ def test_summary_and_mx_diff_on_fake_results():
                                                                           "vs_plain_mxfp4_pct": 3.0}}},
            "parity": {"ok": True, "activations": {"exempt": 0}, "weights": {"exempt": 0}, "y_rel_fro_vs_oracle": 1e-6}}
     sm = bench.summary(out)
-    assert set(sm) == {"cfg4_down_prefill", "cfg2_llama_up", "cfg3_M1", "cfg5_M1", "moe_up_T16", "parity_cfg4"}
+    assert set(sm) == {"cfg4_down_prefill", "cfg2_llama_up", "cfg3_M1", "cfg5_M1", "moe_up_T16", "parity_cfg4",
+                       "flip_llama_up"}
     codes = np.zeros((1, 16), np.uint8)  # one 32-element block
     codes[0, :2] = [0x21, 0x43]
     scales = np.array([[120]], np.uint8)

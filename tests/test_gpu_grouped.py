@@ -105,15 +105,18 @@ def test_device_counts_match_host_counts(mq, name, counts, N, K, dtype):
     x = (torch.randn(T, K, generator=g) * 2).to(torch.bfloat16).cuda()
     host = mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N)
     ws = torch.full((mq.grouped_device_workspace_bytes(T, E, N, K),), 0xFF, dtype=torch.uint8, device="cuda")
-    dev = mq.macaq_w4a4_grouped_linear_device(x, torch.tensor(counts, dtype=dtype, device="cuda"), am, Wq, Ws, N,
-                                              workspace=ws)
-    dev2 = mq.macaq_w4a4_grouped_linear_device(x, torch.tensor(counts, dtype=dtype, device="cuda"), None, Wq, Ws, N)
+    cd = torch.tensor(counts, dtype=dtype, device="cuda")
+    dev = mq.macaq_w4a4_grouped_linear_device(x, cd, am, Wq, Ws, N, workspace=ws)
+    dev2 = mq.macaq_w4a4_grouped_linear_device(x, cd, None, Wq, Ws, N)
+    # an expert capacity at the largest count picks the narrow decode kernels where it can
+    devc = mq.macaq_w4a4_grouped_linear_device(x, cd, am, Wq, Ws, N, capacity=max(counts))
     plain = mq.macaq_w4a4_grouped_linear(x, counts, None, Wq, Ws, N)
     torch.cuda.synchronize()
     assert mq.macaq_device_status() == 0
     assert bool(torch.isfinite(dev.float()).all())
     assert gu.rel_fro(gu.to_np(dev.float()), gu.to_np(host.float())) <= TOL
     assert gu.rel_fro(gu.to_np(dev2.float()), gu.to_np(plain.float())) <= TOL
+    assert gu.rel_fro(gu.to_np(devc.float()), gu.to_np(host.float())) <= TOL
 
 
 def test_device_counts_out_of_range_are_corrected_and_reported(mq):
@@ -132,3 +135,21 @@ def test_device_counts_out_of_range_are_corrected_and_reported(mq):
     # expert 2's count is cut at the 30 rows that remain after expert 0: rows 10..39
     assert gu.rel_fro(gu.to_np(y[:10].float()), gu.to_np(ref[:10].float())) <= TOL
     assert bool(torch.isfinite(y.float()).all())
+
+
+def test_device_counts_above_capacity_are_not_computed(mq):
+    """An expert with more rows than the capacity: its first `capacity` rows are computed, the rest
+    of its rows of y are left as they were, later experts keep their place in x, and MACAQ_ECOUNTS
+    is reported."""
+    N, K = 256, 512
+    Wq, Ws, am = _experts(mq, 3, N, K, seed=13)
+    counts = [5, 12, 7]
+    x = (torch.randn(sum(counts), K) * 2).to(torch.bfloat16).cuda()
+    ref = mq.macaq_w4a4_grouped_linear(x, counts, am, Wq, Ws, N)
+    y = torch.full((sum(counts), N), 7.0, dtype=torch.bfloat16, device="cuda")
+    mq.macaq_w4a4_grouped_linear_device(x, torch.tensor(counts, device="cuda"), am, Wq, Ws, N, capacity=8, y=y)
+    torch.cuda.synchronize()
+    assert mq.macaq_device_status(clear=True) == -8
+    done = list(range(0, 5)) + list(range(5, 13)) + list(range(17, 24))  # expert 1: rows 5..12 of 5..16
+    assert gu.rel_fro(gu.to_np(y[done].float()), gu.to_np(ref[done].float())) <= TOL
+    assert bool((y[13:17] == 7.0).all())
