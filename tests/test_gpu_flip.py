@@ -35,7 +35,8 @@ def _layer(N, K, C, seed):
 
 
 @pytest.mark.parametrize("N,K,C,max_moves", [(300, 1024, 64, 10_000), (130, 1056, 40, 10_000), (64, 512, 33, 0),
-                                             (64, 512, 33, 1), (200, 768, 96, 3)],
+                                             (64, 512, 33, 1), (200, 768, 96, 3),
+                                             (2100, 256, 40, 50)],  # two chunks of rows (2048 + 52)
                          ids=lambda v: str(v))
 def test_flip_refine_matches_oracle(mq, N, K, C, max_moves):
     W, s, xcal = _layer(N, K, C, N + K + C + max_moves)
