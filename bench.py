@@ -319,16 +319,19 @@ def time_eager(fn, steps, warmup, device):
     return e0.elapsed_time(e1) / steps
 
 
-def time_ab(fns, steps, warmup, device, rounds=5):
+def time_ab(fns, steps, warmup, device, rounds=7):
     """ms per call of each fn in `fns` (name -> fn), each captured as a graph of `steps` calls;
-    the graphs are replayed in turn for `rounds` rounds and each fn's median is returned, so a
-    drift of the clock or of the board's power state during the run falls on every fn alike
-    (the comparisons -- overhead against plain MXFP4 -- are differences of a few percent)."""
+    the graphs are replayed in turn for `rounds` rounds, the order rotated every round so that no
+    variant always follows the same one (the board's power state carries over from one replay to
+    the next), and each fn's median is returned, so a drift of the clock or of the power state
+    falls on every fn alike (the comparisons -- overhead against plain MXFP4 -- are differences of
+    a few percent)."""
     loops = {name: GraphLoop(fn, steps, warmup, device) for name, fn in fns.items()}
+    names = list(loops)
     times = {name: [] for name in fns}
-    for _ in range(rounds):
-        for name, g in loops.items():
-            times[name].append(g.time_ms() / steps)
+    for r in range(rounds):
+        for name in names[r % len(names):] + names[:r % len(names)]:
+            times[name].append(loops[name].time_ms() / steps)
     del loops
     return {name: statistics.median(v) for name, v in times.items()}
 
@@ -622,7 +625,7 @@ def prefill_leg(layer, args, peaks):
         "overhead": {"linear_ms": ms_lin, "plain_mxfp4_ms": ms_plain, "gemm_only_ms": ms_gemm,
                      "vs_plain_mxfp4_pct": 100.0 * (ms_lin / ms_plain - 1.0),
                      "vs_gemm_only_pct": 100.0 * (ms_lin / ms_gemm - 1.0),
-                     "method": "medians of 5 alternating graph replays per variant",
+                     "method": "medians of 7 rounds of alternating graph replays per variant, order rotated each round",
                      "transform_quant_ms": ms_xform,
                      "transform_quant_gbs": xform_bytes / (ms_xform * 1e-3) / 1e9},
     }
@@ -720,7 +723,7 @@ def stack_sweep(mq, device, peaks, Ms=(1, 32, 512, 4096), steps=3, warmup=2):
             for K, N, Wq, Ws, am in lin:
                 mq.macaq_mxfp4_linear(xs[K], Wq, Ws, N, y=ys[N], workspace=ws)
 
-        ab = time_ab({"w4a4": w4a4, "plain": plain}, steps, warmup, device, rounds=3)
+        ab = time_ab({"w4a4": w4a4, "plain": plain}, steps, warmup, device, rounds=5)
         ms, ms_plain = ab["w4a4"], ab["plain"]
         flops = sum(2.0 * M * K * N for K, N, *_ in lin)
         nbytes = sum(wls.alg_bytes(wls.Workload("", 5, M, K, N, "normal", 0.0, 1.0)) for K, N, *_ in lin)
