@@ -81,6 +81,14 @@ size_t macaq_scale_bytes(int64_t rows, int64_t K);
 /* Offset of the scale byte of (row r, 32-block kb) in that buffer (-1 if out of range). */
 int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K);
 
+/* Conversions between row-major E8M0 scales, uint8 [rows][K/32] (the layout most MXFP4 producers
+ * write), and the MMA tile layout above (macaq_scale_bytes(rows, K) bytes), on the device, for
+ * callers that quantise activations or weights elsewhere.  To the tile layout, the padded blocks of
+ * real rows and the padded rows are written as 0; back, only the real rows and blocks are written.
+ * Asynchronous on `stream`; MACAQ_EINVAL for a null pointer, MACAQ_ESHAPE as for the other calls. */
+int macaq_scales_to_tiled(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* tiled, void* stream);
+int macaq_scales_to_rowmajor(const uint8_t* tiled, int64_t rows, int64_t K, uint8_t* rowmajor, void* stream);
+
 /* Bytes of scratch macaq_mxfp4_gemm uses for its stream-K schedule on the current device
  * (256 eight-byte flag words and a 128-row fp32 partial-sum slot per CTA of the persistent
  * grid; depends on M and the device's SM count).  The scratch needs no initialisation: a

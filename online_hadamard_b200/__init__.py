@@ -28,7 +28,8 @@ __all__ = [
     "macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_grouped_linear",
     "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian", "macaq_flip_refine",
-    "macaq_w4a4_grouped_linear_device", "grouped_device_workspace_bytes",
+    "macaq_w4a4_grouped_linear_device", "grouped_device_workspace_bytes", "macaq_scales_to_tiled",
+    "macaq_scales_to_rowmajor",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
@@ -41,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "macaq_grouped_workspace_bytes", "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc",
     "macaq_hessian_workspace_bytes", "macaq_calib_hessian", "macaq_flip_refine_workspace_bytes",
     "macaq_flip_refine", "macaq_grouped_device_workspace_bytes", "macaq_w4a4_grouped_linear_device",
+    "macaq_scales_to_tiled", "macaq_scales_to_rowmajor",
 )
 
 MACAQ_OK = 0
@@ -94,13 +96,16 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_flip_refine_workspace_bytes.argtypes = [i64, i64]
         lib.macaq_flip_refine_workspace_bytes.restype = sz
         lib.macaq_flip_refine.argtypes = [p, i64, i64, p, p, p, p, i64, p, p, sz, p]
+        lib.macaq_scales_to_tiled.argtypes = [p, i64, i64, p, p]
+        lib.macaq_scales_to_rowmajor.argtypes = [p, i64, i64, p, p]
         lib.macaq_grouped_device_workspace_bytes.argtypes = [i64, i32, i64, i64]
         lib.macaq_grouped_device_workspace_bytes.restype = sz
         lib.macaq_w4a4_grouped_linear_device.argtypes = [p, i64, p, i32, i32, i64, i64, p, p, p, i64, p, p, sz, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian",
-                     "macaq_flip_refine", "macaq_w4a4_grouped_linear_device"):
+                     "macaq_flip_refine", "macaq_w4a4_grouped_linear_device", "macaq_scales_to_tiled",
+                     "macaq_scales_to_rowmajor"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -185,6 +190,31 @@ def gemm_workspace_bytes(M: int, N: int, K: int, device=None) -> int:
     """Scratch bytes of the GEMM's stream-K schedule on `device` (default: the current one)."""
     with _device(device):
         return int(load_library().macaq_gemm_workspace_bytes(M, N, K))
+
+
+def macaq_scales_to_tiled(rowmajor: torch.Tensor, K: int, tiled=None, stream=None):
+    """Row-major E8M0 scales uint8 [rows, K/32] -> the MMA tile layout (uint8 [scale_bytes(rows, K)])."""
+    rows = rowmajor.shape[0]
+    _need(rowmajor, "rowmajor", torch.uint8, (rows, K // 32))
+    dev = rowmajor.device
+    tiled = torch.empty(scale_bytes(rows, K), dtype=torch.uint8, device=dev) if tiled is None else tiled
+    _need(tiled, "tiled", torch.uint8, min_numel=scale_bytes(rows, K), device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_scales_to_tiled(_ptr(rowmajor), rows, K, _ptr(tiled), _stream(stream, dev)),
+               "macaq_scales_to_tiled")
+    return tiled
+
+
+def macaq_scales_to_rowmajor(tiled: torch.Tensor, rows: int, K: int, rowmajor=None, stream=None):
+    """MMA-tile-layout E8M0 scales -> row-major uint8 [rows, K/32]."""
+    _need(tiled, "tiled", torch.uint8, min_numel=scale_bytes(rows, K))
+    dev = tiled.device
+    rowmajor = torch.empty(rows, K // 32, dtype=torch.uint8, device=dev) if rowmajor is None else rowmajor
+    _need(rowmajor, "rowmajor", torch.uint8, (rows, K // 32), device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_scales_to_rowmajor(_ptr(tiled), rows, K, _ptr(rowmajor), _stream(stream, dev)),
+               "macaq_scales_to_rowmajor")
+    return rowmajor
 
 
 def macaq_calibrate_scale(xcal: torch.Tensor, W: torch.Tensor, s=None, stream=None):

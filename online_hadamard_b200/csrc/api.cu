@@ -50,6 +50,46 @@ extern "C" int64_t macaq_scale_offset(int64_t r, int64_t kb, int64_t K) {
     return scale_offset(r, kb, padded_blocks(K));
 }
 
+namespace macaq {
+
+// One thread per scale byte of the tiled buffer (rows padded to 128, blocks to KBp): row-major
+// [rows][K/32] E8M0 bytes to the MMA tile layout (padded blocks and padded rows written as 0),
+// or back (real rows and blocks only).
+__global__ void scales_layout_kernel(const uint8_t* __restrict__ src, int64_t rows, int64_t K, uint8_t* __restrict__ dst,
+                                     int to_tiled) {
+    const int64_t kb_real = K / 32, kbp = padded_blocks(K);
+    const int64_t prow = (rows + 127) / 128 * 128;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= prow * kbp) return;
+    const int64_t r = i / kbp, kb = i % kbp;
+    const int64_t off = scale_offset(r, kb, kbp);
+    const bool real = r < rows && kb < kb_real;
+    if (to_tiled)
+        dst[off] = real ? src[r * kb_real + kb] : 0;
+    else if (real)
+        dst[r * kb_real + kb] = src[off];
+}
+
+static int launch_scales_layout(const uint8_t* src, int64_t rows, int64_t K, uint8_t* dst, int to_tiled, void* stream) {
+    if (!src || !dst) return MACAQ_EINVAL;
+    if (int st = check_shape(rows, K)) return st;
+    const int64_t n = (rows + 127) / 128 * 128 * padded_blocks(K);
+    scales_layout_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        src, rows, K, dst, to_tiled);
+    return launch_status();
+}
+
+}  // namespace macaq
+
+extern "C" int macaq_scales_to_tiled(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* tiled, void* stream) {
+    return launch_scales_layout(rowmajor, rows, K, tiled, 1, stream);
+}
+
+extern "C" int macaq_scales_to_rowmajor(const uint8_t* tiled, int64_t rows, int64_t K, uint8_t* rowmajor,
+                                        void* stream) {
+    return launch_scales_layout(tiled, rows, K, rowmajor, 0, stream);
+}
+
 extern "C" int macaq_device_status(int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MACAQ_ECUDA;
     int v = 0;

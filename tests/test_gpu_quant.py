@@ -157,3 +157,21 @@ def test_scale_buffer_layout_roundtrip_on_device(mq):
     S = layout.tiled_to_rowmajor(gu.to_np(As), 200, 512)
     expect = np.array([[(r + 3 * b) % 40 - 20 + 127 - 2 for b in range(16)] for r in range(200)])
     assert np.array_equal(S, expect)
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (200, 1056), (300, 4096), (129, 96)], ids=str)
+def test_scale_layout_conversions(mq, rows, K):
+    """Row-major E8M0 scales to the MMA tile layout and back, against the documented index map
+    (tests/layout.py), padded blocks and rows zero; and the quantiser's own scales round-trip."""
+    rng = np.random.default_rng(rows + K)
+    S = rng.integers(0, 255, (rows, K // 32)).astype(np.uint8)
+    tiled = mq.macaq_scales_to_tiled(torch.from_numpy(S).cuda(), K)
+    back = mq.macaq_scales_to_rowmajor(tiled, rows, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.to_np(tiled), layout.rowmajor_to_tiled(S, rows, K))
+    assert np.array_equal(gu.to_np(back), S)
+    x = (torch.randn(rows, K) * 3).to(torch.bfloat16).cuda()
+    Aq, As = mq.macaq_act_quant_plain(x)
+    rm = mq.macaq_scales_to_rowmajor(As, rows, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.to_np(rm), layout.tiled_to_rowmajor(gu.to_np(As), rows, K))
