@@ -186,3 +186,46 @@ def test_fault_injection_hook_only_in_the_test_build():
     fault = ctypes.CDLL(b.build_fault_library())
     assert hasattr(fault, "macaq_test_owner_tag_offset")
     assert not hasattr(mq.load_library(), "macaq_test_owner_tag_offset")
+
+
+def test_validation_of_the_offline_and_grouped_device_calls():
+    """Flip-Refinement, the calibration Hessian, the device-count grouped linear and the scale-layout
+    conversions refuse bad arguments before any CUDA call (fake pointers are never used)."""
+    P = ctypes.c_void_p
+    lib = mq.load_library()
+    # sizes: pure host arithmetic
+    assert lib.macaq_hessian_workspace_bytes(64, 256) == 64 * 256 * 4
+    assert lib.macaq_hessian_workspace_bytes(64, 200) == 0
+    assert lib.macaq_flip_refine_workspace_bytes(300, 1024) == 300 * 1024 * 12
+    assert lib.macaq_flip_refine_workspace_bytes(5000, 1024) == 2048 * 1024 * 12  # one chunk of rows
+    assert lib.macaq_flip_refine_workspace_bytes(4, 12320) == 0                  # K above the limit
+    assert lib.macaq_grouped_device_workspace_bytes(128, 129, 256, 512) == 0      # more than 128 experts
+    assert lib.macaq_grouped_device_workspace_bytes(128, 16, 200, 512) == 0       # N % 128 != 0
+    assert lib.macaq_grouped_device_workspace_bytes(128, 16, 256, 512) > 0
+    # macaq_calib_hessian(xcal, C, K, act_mult, Hs, ws, ws_bytes, stream)
+    assert _call("macaq_calib_hessian", None, 64, 256, P(FAKE), P(FAKE), P(FAKE), 1 << 20, None) == -1
+    assert _call("macaq_calib_hessian", P(FAKE), 64, 200, P(FAKE), P(FAKE), P(FAKE), 1 << 20, None) == -2
+    assert _call("macaq_calib_hessian", P(FAKE), 64, 256, P(MIS), P(FAKE), P(FAKE), 1 << 20, None) == -3
+    assert _call("macaq_calib_hessian", P(FAKE), 64, 256, P(FAKE), P(FAKE), P(FAKE), 100, None) == -6
+    # macaq_flip_refine(W, N, K, s, Hs, Wq, Ws, max_moves, moves, ws, ws_bytes, stream)
+    ok = (P(FAKE), 300, 1024, P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    assert _call("macaq_flip_refine", *ok, -1, None, P(FAKE), 1 << 30, None) == -1        # negative budget
+    assert _call("macaq_flip_refine", None, *ok[1:], 8, None, P(FAKE), 1 << 30, None) == -1
+    assert _call("macaq_flip_refine", P(FAKE), 300, 12320, *ok[3:], 8, None, P(FAKE), 1 << 30, None) == -2
+    assert _call("macaq_flip_refine", *ok, 8, P(MIS), P(FAKE), 1 << 30, None) == -3       # moves misaligned
+    assert _call("macaq_flip_refine", *ok, 8, None, P(FAKE), 1000, None) == -6            # workspace too small
+    # macaq_w4a4_grouped_linear_device(x, T, counts, counts_bytes, E, capacity, K, act_mult, Wq, Ws, N, y, ws,
+    #                                  ws_bytes, stream)
+    g = lambda **kw: _call("macaq_w4a4_grouped_linear_device", kw.get("x", P(FAKE)), kw.get("T", 128),
+                           kw.get("counts", P(FAKE)), kw.get("cb", 4), kw.get("E", 16), 0, kw.get("K", 512),
+                           P(FAKE), P(FAKE), P(FAKE), kw.get("N", 256), P(FAKE), P(FAKE), kw.get("wsb", 1 << 30),
+                           None)
+    assert g(counts=None) == -1
+    assert g(cb=3) == -1
+    assert g(E=129) == -2 and g(E=0) == -2
+    assert g(N=200) == -2 and g(K=48) == -2 and g(T=0) == -2
+    assert g(counts=P(FAKE + 2)) == -3                                                     # int32 counts misaligned
+    assert g(wsb=1000) == -6
+    # layout conversions
+    assert _call("macaq_scales_to_tiled", None, 4, 64, P(FAKE), None) == -1
+    assert _call("macaq_scales_to_rowmajor", P(FAKE), 4, 48, P(FAKE), None) == -2
