@@ -652,7 +652,8 @@ def summary(out):
     for k, v in st.items():
         if k.startswith("M"):
             sm["cfg5_" + k] = {"ms": r(v["w4a4_ms"]), "roof": r(v["linear_roofline_frac"]),
-                               "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2)}
+                               "ovh_plain_pct": r(v["vs_plain_mxfp4_pct"], 2),
+                               "unstacked_ms": r(v["w4a4_one_linear_at_a_time_ms"])}
     for k, v in (sec.get("qwen3_moe_grouped") or {}).items():
         if isinstance(v, dict):
             sm["moe_" + k] = {"us": r(v["ms"] * 1e3), "roof": r(v["linear_roofline_frac"]),
@@ -690,50 +691,86 @@ def profile_kernels(name):
     print(f"profiled {wl.name} M={wl.M} K={wl.K} N={wl.N}")
 
 
+# Layers of a decoder block that read the same activations: run as one stacked call.
+STACK_GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))
+
+
 def stack_sweep(mq, device, peaks, Ms=(1, 32, 512, 4096), steps=3, warmup=2):
     """The 64-layer Qwen3-32B-shaped linear stack (q, k, v, o, gate, up, down per layer): each
     linear's weights and calibration batch are drawn on the device, s is calibrated and W folded
     by the library, and the fp32 weights are freed before the next linear, so only the 16.6 GB
-    of MXFP4 weights stay resident.  Per M, all 448 linears run back to back in one CUDA graph,
-    as W4A4 linears and as plain-MXFP4 linears; the summed times give the transform's overhead."""
-    lin = []
+    of MXFP4 weights stay resident.  The layers reading the same activations (q, k, v; gate, up)
+    are folded into slices of one stacked buffer each.  Per M, all 448 linears run back to back in
+    one CUDA graph three ways: W4A4 with the shared-input layers stacked (macaq_w4a4_linear_multi:
+    q/k/v and gate/up each one quantiser and one GEMM launch), plain MXFP4 stacked the same way
+    (the overhead's baseline), and W4A4 one linear at a time."""
+    dims = {name: (K, N) for name, K, N in wls.QWEN_STACK_LINEARS}
+    groups = []  # per (layer, group): K, Ns, stacked Wq, Ws, act_mult [G, K]
     for layer in range(64):
-        for name, K, N in wls.QWEN_STACK_LINEARS:
-            wl = wls.stack_layer(layer, name, 1)
-            W = wls.make_w_device(wl, device)
-            s = mq.macaq_calibrate_scale(wls.make_x_device(wl, wls.CALIB_TOKENS, device, tensor_id=2), W)
-            Wq, Ws, am = mq.macaq_fold_weights(W, s)
-            del W
-            lin.append((K, N, Wq, Ws, am))
+        for names in STACK_GROUPS:
+            K = dims[names[0]][0]
+            Ns = [dims[n][1] for n in names]
+            Wq = torch.empty(sum(Ns), K // 2, dtype=torch.uint8, device=device)
+            sb = [mq.scale_bytes(N, K) for N in Ns]
+            Ws = torch.empty(sum(sb), dtype=torch.uint8, device=device)
+            am = torch.empty(len(names), K, dtype=torch.float32, device=device)
+            n0 = b0 = 0
+            for g, name in enumerate(names):
+                wl = wls.stack_layer(layer, name, 1)
+                W = wls.make_w_device(wl, device)
+                s = mq.macaq_calibrate_scale(wls.make_x_device(wl, wls.CALIB_TOKENS, device, tensor_id=2), W)
+                mq.macaq_fold_weights(W, s, Wq=Wq[n0:n0 + Ns[g]], Ws=Ws[b0:b0 + sb[g]], act_mult=am[g])
+                del W
+                n0 += Ns[g]
+                b0 += sb[g]
+            groups.append((K, Ns, Wq, Ws, am, sb))
     torch.cuda.empty_cache()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    res = {"layers": 64, "linears": len(lin), "weights_gb": sum(q.numel() + t.numel() for _, _, q, t, _ in lin) / 1e9}
+    res = {"layers": 64, "linears": sum(len(g[1]) for g in groups),
+           "weights_gb": sum(q.numel() + t.numel() for _, _, q, t, _, _ in groups) / 1e9,
+           "stacked": "+".join("/".join(n) for n in STACK_GROUPS)}
     for M in Ms:
         xs = {K: wls.make_x_device(wls.stack_layer(0, name, M), M, device)
               for name, K, _ in wls.QWEN_STACK_LINEARS}
-        ys = {N: torch.empty(M, N, dtype=torch.bfloat16, device=device) for _, _, N in wls.QWEN_STACK_LINEARS}
-        ws = torch.empty(max(mq.linear_workspace_bytes(M, N, K) for _, K, N in wls.QWEN_STACK_LINEARS),
+        ys = {tuple(Ns): torch.empty(M, sum(Ns), dtype=torch.bfloat16, device=device) for _, Ns, *_ in groups}
+        ws = torch.empty(max(max(mq.linear_multi_workspace_bytes(M, len(Ns), K) for K, Ns, *_ in groups),
+                             max(mq.linear_workspace_bytes(M, N, K) for _, K, N in wls.QWEN_STACK_LINEARS)),
                          dtype=torch.uint8, device=device)
+        # the one-linear-at-a-time variant's operands: views into the stacked buffers
+        singles = []
+        for K, Ns, Wq, Ws, am, sb in groups:
+            n0 = b0 = 0
+            for g, N in enumerate(Ns):
+                singles.append((K, N, Wq[n0:n0 + N], Ws[b0:b0 + sb[g]], am[g]))
+                n0 += N
+                b0 += sb[g]
+        y1 = {N: torch.empty(M, N, dtype=torch.bfloat16, device=device) for _, _, N in wls.QWEN_STACK_LINEARS}
 
         def w4a4(i):
-            for K, N, Wq, Ws, am in lin:
-                mq.macaq_w4a4_linear(xs[K], am, Wq, Ws, N, y=ys[N], workspace=ws)
+            for K, Ns, Wq, Ws, am, _ in groups:
+                mq.macaq_w4a4_linear_multi(xs[K], am, Wq, Ws, Ns, y=ys[tuple(Ns)], workspace=ws)
 
         def plain(i):
-            for K, N, Wq, Ws, am in lin:
-                mq.macaq_mxfp4_linear(xs[K], Wq, Ws, N, y=ys[N], workspace=ws)
+            for K, Ns, Wq, Ws, _, _ in groups:
+                mq.macaq_w4a4_linear_multi(xs[K], None, Wq, Ws, Ns, y=ys[tuple(Ns)], workspace=ws)
 
-        ab = time_ab({"w4a4": w4a4, "plain": plain}, steps, warmup, device, rounds=5)
+        def unstacked(i):
+            for K, N, Wq, Ws, am in singles:
+                mq.macaq_w4a4_linear(xs[K], am, Wq, Ws, N, y=y1[N], workspace=ws)
+
+        ab = time_ab({"w4a4": w4a4, "plain": plain, "unstacked": unstacked}, steps, warmup, device, rounds=5)
         ms, ms_plain = ab["w4a4"], ab["plain"]
-        flops = sum(2.0 * M * K * N for K, N, *_ in lin)
-        nbytes = sum(wls.alg_bytes(wls.Workload("", 5, M, K, N, "normal", 0.0, 1.0)) for K, N, *_ in lin)
+        flops = sum(2.0 * M * K * N for K, Ns, *_ in groups for N in Ns)
+        nbytes = sum(wls.alg_bytes(wls.Workload("", 5, M, K, N, "normal", 0.0, 1.0)) for K, Ns, *_ in groups
+                     for N in Ns)
         t_roof = max(flops / (fp4_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
         res[f"M{M}"] = {"w4a4_ms": ms, "plain_mxfp4_ms": ms_plain, "vs_plain_mxfp4_pct": 100.0 * (ms / ms_plain - 1.0),
+                        "w4a4_one_linear_at_a_time_ms": ab["unstacked"],
                         "tflops": flops / (ms * 1e-3) / 1e12, "gbs": nbytes / (ms * 1e-3) / 1e9,
                         "linear_roofline_frac": t_roof / (ms * 1e-3)}
-        del xs, ys, ws
+        del xs, ys, ws, singles, y1
         torch.cuda.empty_cache()
-    del lin
+    del groups
     torch.cuda.empty_cache()
     return res
 

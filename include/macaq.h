@@ -3,11 +3,10 @@
  * linear layer on NVIDIA B200 (sm_100a).
  *
  * Method: "MACaQ: Fast, Model Agnostic Calibrated Quantization for Low-Precision Weights
- * and Activations" (arXiv 2611.10649), Abstract: every linear layer is treated on its
- * own; a per-channel scale and a block-Hadamard transform are applied online to the
- * layer's activations while the corresponding inverse transforms are absorbed into the
- * layer's weights; weights and activations are MXFP4 (W4A4), the weights rounded to
- * nearest.  The pages leave the details open; this library fixes them as follows.
+ * and Activations" (arXiv 2611.10649), Abstract: no linear layer depends on another; at
+ * inference the activations of a layer are scaled channel by channel and rotated by a
+ * block Hadamard, and the inverse of both is folded into the same layer's weights; both
+ * operands are MXFP4 (W4A4), the weights rounded to nearest.  The pages leave the details open; this library fixes them as follows.
  *
  *   Notation.  x is bf16 [M][K] row-major, W is fp32 [N][K] row-major (y = x W^T, the
  *   nn.Linear layout), s is fp32 [K] with s_k > 0 finite.  c = 1/sqrt(32).
@@ -117,8 +116,8 @@ int macaq_calibrate_scale(const uint16_t* xcal, int64_t C, const float* W, int64
                           float* s, void* stream);
 
 /*
- * macaq_fold_weights -- offline weight preparation (Abstract: "absorbing the corresponding
- * inverse transforms into its weights"; weights quantised round-to-nearest).
+ * macaq_fold_weights -- offline weight preparation (Abstract: the inverse of the activation
+ * transforms is folded into the layer's weights, which are then rounded to nearest).
  *   W        in   fp32 [N][K]
  *   s        in   fp32 [K], every s_k finite and > 0 (else MACAQ_EINVAL, nothing written)
  *   Wq       out  MXFP4 codes [N][K/2] of W' = W diag(s) H_bd / sqrt(32)
@@ -131,9 +130,9 @@ int macaq_fold_weights(const float* W, int64_t N, int64_t K, const float* s, uin
                        uint8_t* Ws, float* act_mult, void* stream);
 
 /*
- * macaq_act_transform_quant -- the online activation transform (Abstract: "a per-channel
- * scale and a block-Hadamard transform online to each layer's activations") followed by
- * MXFP4 quantisation (the A4 of W4A4).
+ * macaq_act_transform_quant -- the online activation transform (Abstract: the layer's
+ * activations are scaled per channel and rotated by a block Hadamard at inference time)
+ * followed by MXFP4 quantisation (the A4 of W4A4).
  *   x        in   bf16 bit patterns [M][K]
  *   act_mult in   fp32 [K] (from macaq_fold_weights)
  *   Aq       out  MXFP4 codes [M][K/2]
@@ -144,8 +143,8 @@ int macaq_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const flo
 
 /*
  * macaq_w4a4_linear -- the layer's forward pass, y = x W^T computed as
- * MXFP4(x diag(act_mult) H) . MXFP4(W')^T (Abstract; the 2.3% end-to-end overhead over
- * plain MXFP4 quoted there is for this online transform): the activation transform and
+ * MXFP4(x diag(act_mult) H) . MXFP4(W')^T (Abstract; the 2.3 % end-to-end cost the pages give
+ * against MXFP4 without transforms is that of this online transform): the activation transform and
  * MXFP4 quantisation kernel writes the activations' codes and scales into the workspace,
  * then the block-scaled MXFP4 x MXFP4 GEMM (launched as a programmatic dependent of it)
  * contracts them on the tensor cores with fp32 accumulation and rounds y to bf16 (RNE).
@@ -187,6 +186,35 @@ int macaq_mxfp4_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* W
 int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq,
                      const uint8_t* Ws, int64_t N, int64_t K, void* y, int y_is_fp32,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * macaq_w4a4_linear_multi -- G linear layers on the same activations x, e.g. the q, k and v
+ * projections of an attention block or the gate and up projections of an MLP.  Each is its own
+ * layer with its own per-channel scale and folded weights (the method is layer-local, Abstract),
+ * so x is transformed and quantised once per layer, in ONE launch; then, for M <= 128, ONE
+ * swap-AB GEMM runs over the layers' weights stacked by rows, each 128-row weight tile against
+ * its own layer's activation tile (above 128 tokens, one GEMM per layer).
+ *   x         in   bf16 [M][K]
+ *   act_mult  in   fp32 [G][K], layer g's multipliers from macaq_fold_weights at g*K; NULL: plain
+ *                  MXFP4 of x, quantised once and shared (the "pure MXFP4" baseline)
+ *   Wq, Ws    in   the layers' folded weights stacked in order g = 0..G-1: codes [sum N][K/2],
+ *                  scales the G buffers of macaq_scale_bytes(N[g], K) bytes one after another
+ *   N         in   HOST int64 [G], 1 <= G <= 128, every N[g] a positive multiple of 128
+ *   y         out  bf16 [M][sum N]: layer g's outputs in columns N[0] + .. + N[g-1] onwards
+ *   workspace in   at least macaq_linear_multi_workspace_bytes(M, G, K) bytes.  With Mp = M
+ *                  rounded up to a multiple of 128, layer g's activation codes [M][K/2] are left
+ *                  at byte g*Mp*K/2 and their scales (MMA tile layout) at byte A + g *
+ *                  macaq_scale_bytes(Mp, K), A = G*Mp*K/2 rounded up to 256 (act_mult NULL: the
+ *                  one shared set at g = 0); the GEMM's stream-K scratch follows.  Other bytes
+ *                  are unspecified on return; calls sharing it must be stream-ordered
+ * Layer g's activation codes and scales equal those of macaq_act_transform_quant(x, act_mult +
+ * g*K) bit for bit, and its y columns equal macaq_w4a4_linear's within the GEMM tolerance (the
+ * stacked launch may split the K steps differently).  MACAQ_ESHAPE for G or an N[g] out of range.
+ */
+size_t macaq_linear_multi_workspace_bytes(int64_t M, int G, int64_t K);
+int macaq_w4a4_linear_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult,
+                            const uint8_t* Wq, const uint8_t* Ws, const int64_t* N, uint16_t* y,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * macaq_w4a4_grouped_linear -- a grouped (mixture-of-experts) W4A4 linear: E experts, each its
@@ -272,8 +300,8 @@ int macaq_w4a4_linear_noalloc(const uint16_t* x, int64_t M, int64_t K, const flo
                               void* stream);
 
 /*
- * Flip-Refinement (Abstract: "a Hessian-aware coordinate-descent procedure that greedily moves
- * individual FP4 codes to adjacent representable values", improving on round-to-nearest).  An
+ * Flip-Refinement (Abstract: a greedy coordinate descent, weighted by the Hessian, that shifts
+ * single FP4 codes to a neighbouring grid value, starting from round-to-nearest).  An
  * offline step between macaq_fold_weights and inference; the pages give no more, and this library
  * reads it as follows (details in csrc/flip.cu):
  *   objective of weight row n:  L_n = (q_n - v_n) Hs (q_n - v_n)^T, q_n the decoded codes, v_n the

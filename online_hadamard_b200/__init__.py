@@ -29,7 +29,7 @@ __all__ = [
     "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_w4a4_grouped_linear",
     "grouped_workspace_bytes", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian", "macaq_flip_refine",
     "macaq_w4a4_grouped_linear_device", "grouped_device_workspace_bytes", "macaq_scales_to_tiled",
-    "macaq_scales_to_rowmajor",
+    "macaq_scales_to_rowmajor", "macaq_w4a4_linear_multi", "linear_multi_workspace_bytes",
     "macaq_device_status", "status_str", "EXPORTED_SYMBOLS",
 ]
 
@@ -42,7 +42,8 @@ EXPORTED_SYMBOLS = (
     "macaq_grouped_workspace_bytes", "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc",
     "macaq_hessian_workspace_bytes", "macaq_calib_hessian", "macaq_flip_refine_workspace_bytes",
     "macaq_flip_refine", "macaq_grouped_device_workspace_bytes", "macaq_w4a4_grouped_linear_device",
-    "macaq_scales_to_tiled", "macaq_scales_to_rowmajor",
+    "macaq_scales_to_tiled", "macaq_scales_to_rowmajor", "macaq_linear_multi_workspace_bytes",
+    "macaq_w4a4_linear_multi",
 )
 
 MACAQ_OK = 0
@@ -101,11 +102,14 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.macaq_grouped_device_workspace_bytes.argtypes = [i64, i32, i64, i64]
         lib.macaq_grouped_device_workspace_bytes.restype = sz
         lib.macaq_w4a4_grouped_linear_device.argtypes = [p, i64, p, i32, i32, i64, i64, p, p, p, i64, p, p, sz, p]
+        lib.macaq_linear_multi_workspace_bytes.argtypes = [i64, i32, i64]
+        lib.macaq_linear_multi_workspace_bytes.restype = sz
+        lib.macaq_w4a4_linear_multi.argtypes = [p, i64, i64, i32, p, p, p, p, p, p, sz, p]
         for name in ("macaq_calibrate_scale", "macaq_fold_weights", "macaq_act_transform_quant", "macaq_act_quant_plain",
                      "macaq_mxfp4_gemm", "macaq_w4a4_linear", "macaq_mxfp4_linear", "macaq_device_status",
                      "macaq_w4a4_grouped_linear", "macaq_w4a4_linear_noalloc", "macaq_calib_hessian",
                      "macaq_flip_refine", "macaq_w4a4_grouped_linear_device", "macaq_scales_to_tiled",
-                     "macaq_scales_to_rowmajor"):
+                     "macaq_scales_to_rowmajor", "macaq_w4a4_linear_multi"):
             getattr(lib, name).restype = i32
         if path is None:
             _lib = lib
@@ -347,6 +351,43 @@ def macaq_mxfp4_linear(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: i
     with torch.cuda.device(dev):
         _check(load_library().macaq_mxfp4_linear(_ptr(x), M, K, _ptr(Wq), _ptr(Ws), N, _ptr(y), _ptr(workspace),
                                                  workspace.numel(), _stream(stream, dev)), "macaq_mxfp4_linear")
+    return y
+
+
+def linear_multi_workspace_bytes(M: int, G: int, K: int, device=None) -> int:
+    """Scratch bytes macaq_w4a4_linear_multi needs for G linears on M tokens (default device: the
+    current one; the size depends on its SM count)."""
+    with _device(device):
+        return int(load_library().macaq_linear_multi_workspace_bytes(M, G, K))
+
+
+def macaq_w4a4_linear_multi(x: torch.Tensor, act_mult, Wq: torch.Tensor, Ws: torch.Tensor, Ns, y=None,
+                            workspace=None, stream=None):
+    """G linears on the same x [M, K] bf16 (the q, k and v projections, or gate and up), each its own
+    folded layer: act_mult fp32 [G, K] (torch.stack of the folds' multipliers; None: plain MXFP4),
+    Wq [sum Ns, K/2] and Ws (torch.cat of the folds' codes and scales, in the same order), Ns the
+    output features of each (multiples of 128).  Returns y bf16 [M, sum Ns]: linear g's outputs in
+    columns sum(Ns[:g]) .. sum(Ns[:g + 1]) - 1."""
+    import numpy as np
+    M, K = x.shape
+    n = np.ascontiguousarray(np.asarray(list(Ns), dtype=np.int64))
+    G, Nt = len(n), int(n.sum())
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    if act_mult is not None:
+        _need(act_mult, "act_mult", torch.float32, (G, K), device=dev)
+    _need(Wq, "Wq", torch.uint8, (Nt, K // 2), device=dev)
+    _need(Ws, "Ws", torch.uint8, min_numel=sum(scale_bytes(int(v), K) for v in n), device=dev)
+    y = torch.empty(M, Nt, dtype=torch.bfloat16, device=dev) if y is None else y
+    _need(y, "y", torch.bfloat16, (M, Nt), device=dev)
+    need = linear_multi_workspace_bytes(M, G, K, dev)
+    workspace = torch.empty(need, dtype=torch.uint8, device=dev) if workspace is None else workspace
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check(load_library().macaq_w4a4_linear_multi(_ptr(x), M, K, G, _ptr(act_mult), _ptr(Wq), _ptr(Ws),
+                                                      ctypes.c_void_p(n.ctypes.data), _ptr(y), _ptr(workspace),
+                                                      workspace.numel(), _stream(stream, dev)),
+               "macaq_w4a4_linear_multi")
     return y
 
 

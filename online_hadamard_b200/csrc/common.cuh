@@ -54,6 +54,16 @@ struct GroupTable {
 
 struct NoGroups {};
 
+// Several linears on the same activations (the q, k and v projections of a layer, or gate and up),
+// each with its own per-channel scale and folded weights, run as one GEMM over their weights stacked
+// by rows: weight tile t (128 rows) belongs to linear group_of(tile_start, groups, t), whose
+// activation codes (x transformed with that linear's multipliers) start at row a_row of the codes.
+struct SharedActGroups {
+    int groups;
+    int tile_start[kMaxGroups + 1];  // first 128-row weight tile of linear e; [groups] = all tiles
+    int a_row[kMaxGroups];           // first row of linear e's activation codes
+};
+
 // The grouped quantiser's threads: expert e's tokens split into runs of `rpg` rows, its runs
 // numbered from run_start[e]; run_start[E] = all runs (padding rows get no thread).
 struct RowRuns {

@@ -1,9 +1,9 @@
 // flip.cu -- Flip-Refinement of the folded MXFP4 weight codes, and the calibration Hessian it uses.
 //
 // "MACaQ: Fast, Model Agnostic Calibrated Quantization for Low-Precision Weights and
-// Activations", Abstract: to improve over round-to-nearest, Flip-Refinement is a Hessian-aware
-// coordinate-descent procedure that greedily moves individual FP4 codes to adjacent
-// representable values.  The pages say no more; this library reads it as follows.
+// Activations", Abstract: Flip-Refinement starts from the round-to-nearest codes and runs a greedy
+// coordinate descent, weighted by the Hessian, in which a step shifts one FP4 code to a
+// neighbouring grid value.  The pages say no more; this library reads it as follows.
 //   - It refines one layer's folded weight codes (macaq_fold_weights: round to nearest), keeping
 //     every E8M0 block scale: only code nibbles change.
 //   - Objective of output row n: L_n = (q_n - v_n) Hs (q_n - v_n)^T, the layer's output error on a

@@ -54,6 +54,8 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
 int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
                                     uint8_t* As, const DeviceGroups& dg, cudaStream_t stream);
 int64_t device_groups_rpg(int64_t T, int E, int64_t K);
+int launch_act_transform_quant_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult,
+                                     int64_t seg_rows, uint8_t* Aq, uint8_t* As, cudaStream_t stream);
 
 constexpr int kBM = 128;           // MMA M
 constexpr int kStageK = 256;       // K elements per stage
@@ -435,6 +437,7 @@ struct TileRef {
 
 template <int BN, bool SWAP, bool GROUPED, class GT>
 __device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& groups, int tile) {
+    static_assert(SWAP || !std::is_same<GT, SharedActGroups>::value, "stacked linears run swap-AB");
     TileRef t;
     if constexpr (!GROUPED) {
         const int pt = tile % prm.num_p_tiles, qt = tile / prm.num_p_tiles;
@@ -444,6 +447,11 @@ __device__ __forceinline__ TileRef tile_ref(const GemmParams& prm, const GT& gro
         t.y_q = t.q_row;
         t.p_end = prm.p_rows;
         t.q_end = prm.q_rows;
+        if constexpr (std::is_same<GT, SharedActGroups>::value) {
+            // stacked linears on one x (swap-AB: P = the stacked weights): the activation tile is
+            // the one transformed for the linear this weight tile belongs to
+            t.q_row += groups.a_row[group_of(groups.tile_start, groups.groups, pt)];
+        }
     } else {
         const GroupTable& gt = group_table(groups);
         const int e = group_of(gt.tile_start, gt.groups, tile);
@@ -1186,6 +1194,7 @@ struct GemmOperands {
     void* y;
     int64_t ldy;
     int y_fp32;
+    int64_t q_map_rows = 0;  // rows of Q's codes and scales if more than q_rows (stacked linears)
 };
 
 // Scratch of the stream-K schedule (nullptr: data-parallel schedule only).
@@ -1227,10 +1236,11 @@ template <int BN, int STAGES, bool SWAP, class GT = NoGroups>
 static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream_t stream, bool pdl,
                        const GT& groups = GT{}, const GroupedShape* gs = nullptr) {
     using Cfg = TileCfg<BN>;
-    constexpr bool GROUPED = !std::is_same<GT, NoGroups>::value;
-    if (GROUPED && !kernel_attributes<BN, STAGES, SWAP, GROUPED, GT>()) return MACAQ_ECUDA;
+    constexpr bool GROUPED = std::is_same<GT, GroupTable>::value || std::is_same<GT, DeviceGroups>::value;
+    if (!std::is_same<GT, NoGroups>::value && !kernel_attributes<BN, STAGES, SWAP, GROUPED, GT>()) return MACAQ_ECUDA;
+    const int64_t q_map_rows = op.q_map_rows > op.q_rows ? op.q_map_rows : op.q_rows;
     CUtensorMap mp, mq;
-    if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, op.q_rows, op.K, BN))
+    if (!make_codes_map(&mp, op.pq, op.p_rows, op.K, kBM) || !make_codes_map(&mq, op.qq, q_map_rows, op.K, BN))
         return MACAQ_ECUDA;
     GemmParams prm{};
     prm.sf_p = op.ps;
@@ -1245,7 +1255,7 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     prm.num_p_tiles = static_cast<int>((op.p_rows + kBM - 1) / kBM);
     prm.num_q_tiles = static_cast<int>((op.q_rows + BN - 1) / BN);
     prm.num_k_tiles = static_cast<int>((op.K + kStageK - 1) / kStageK);
-    prm.q_row_blocks = static_cast<int>((op.q_rows + 127) / 128);
+    prm.q_row_blocks = static_cast<int>((q_map_rows + 127) / 128);
 
     const int ctas = grid_ctas<BN, STAGES, SWAP>();
     if (ctas < 1) return MACAQ_ECUDA;
@@ -1285,14 +1295,9 @@ static int launch_gemm(const GemmOperands& op, const GemmScratch& ws, cudaStream
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if constexpr (GROUPED) {
-        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP, true, GT>, mp, mq, my, prm, groups) !=
-            cudaSuccess)
-            return MACAQ_ECUDA;
-    } else {
-        if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP>, mp, mq, my, prm, NoGroups{}) != cudaSuccess)
-            return MACAQ_ECUDA;
-    }
+    if (cudaLaunchKernelEx(&cfg, mxf4_gemm_kernel<BN, STAGES, SWAP, GROUPED, GT>, mp, mq, my, prm, groups) !=
+        cudaSuccess)
+        return MACAQ_ECUDA;
     return launch_status();
 }
 
@@ -1440,17 +1445,20 @@ size_t gemm_workspace_bytes(int64_t M) {
     });
 }
 
-// y[M][N] = dec(A) dec(W)^T.  Small M runs swap-AB (weights on the MMA M side).
+// y[M][N] = dec(A) dec(W)^T, row m of y at y + m * ldy elements (ldy = 0: N).  Small M runs
+// swap-AB (weights on the MMA M side).
 int run_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint8_t* Wq, const uint8_t* Ws,
-                   int64_t N, int64_t K, void* y, int y_fp32, const GemmScratch& ws, cudaStream_t stream, bool pdl) {
+                   int64_t N, int64_t K, void* y, int y_fp32, const GemmScratch& ws, cudaStream_t stream, bool pdl,
+                   int64_t ldy = 0) {
+    if (ldy == 0) ldy = N;
     if (use_pairs(M)) {
-        const GemmOperands op{Aq, As, Wq, Ws, M, N, K, y, N, y_fp32};
+        const GemmOperands op{Aq, As, Wq, Ws, M, N, K, y, ldy, y_fp32};
         return launch_gemm_pair(op, ws, gemm_pairs(), stream, pdl);
     }
     return with_config(M, [&](auto bn, auto st, auto sw) -> int {
         constexpr bool kSwap = decltype(sw)::value;
-        const GemmOperands op = kSwap ? GemmOperands{Wq, Ws, Aq, As, N, M, K, y, N, y_fp32}
-                                      : GemmOperands{Aq, As, Wq, Ws, M, N, K, y, N, y_fp32};
+        const GemmOperands op = kSwap ? GemmOperands{Wq, Ws, Aq, As, N, M, K, y, ldy, y_fp32}
+                                      : GemmOperands{Aq, As, Wq, Ws, M, N, K, y, ldy, y_fp32};
         return launch_gemm<decltype(bn)::value, decltype(st)::value, kSwap>(op, ws, stream, pdl);
     });
 }
@@ -1488,6 +1496,77 @@ int run_linear(const uint16_t* x, int64_t M, int64_t K, const float* act_mult, c
     if (rc) return rc;
     const GemmScratch ws{gemm_scratch ? l.gemm : nullptr, gemm_scratch ? l.gemm_bytes : 0};
     return run_mxfp4_gemm(l.Aq, l.As, M, Wq, Ws, N, K, y, 0, ws, st, true);
+}
+
+// Several linears on one x (the q, k and v projections, or gate and up), each with its own
+// multipliers and folded weights, stacked by rows: Wq / Ws hold linear g's N[g] rows after those of
+// the linears before it, and y [M][sum N] holds its outputs in the matching column block.  The
+// workspace holds G segments of activation codes and scales, one per linear, each of whole
+// 128-row blocks (plain MXFP4 of x: one segment, shared), then the GEMM's stream-K scratch.
+size_t grouped_activation_bytes(int64_t padded_rows, int64_t K);
+
+struct MultiWorkspace {
+    uint8_t *Aq, *As, *gemm;
+    size_t gemm_bytes, bytes;
+    int64_t seg_rows;  // rows per linear's segment (a multiple of 128)
+};
+
+static MultiWorkspace multi_workspace_layout(void* base, int64_t M, int G, int64_t K) {
+    MultiWorkspace l;
+    l.seg_rows = (M + 127) / 128 * 128;
+    const int64_t P = G * l.seg_rows;
+    const size_t act = grouped_activation_bytes(P, K);
+    l.Aq = static_cast<uint8_t*>(base);
+    l.As = l.Aq + round256(static_cast<size_t>(P * (K / 2)));
+    l.gemm = l.Aq + act;
+    l.gemm_bytes = gemm_workspace_bytes(M);
+    l.bytes = act + l.gemm_bytes;
+    return l;
+}
+
+// One quantiser launch for all G linears; then, up to 128 tokens, ONE swap-AB GEMM over the
+// stacked weights (each 128-row weight tile paired with its own linear's activation tile), so the
+// small k / v weights share the grid with the rest instead of each running on a few SMs; above
+// 128 tokens one GEMM per linear, each into its column block of y.
+static int run_linear_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult, const uint8_t* Wq,
+                            const uint8_t* Ws, const int64_t* N, int64_t n_total, uint16_t* y,
+                            const MultiWorkspace& l, cudaStream_t st) {
+    const int64_t seg = act_mult ? l.seg_rows : 0;  // row offset between the linears' segments
+    const int rc = act_mult ? launch_act_transform_quant_multi(x, M, K, G, act_mult, l.seg_rows, l.Aq, l.As, st)
+                            : launch_act_quant_plain(x, M, K, l.Aq, l.As, st);
+    if (rc) return rc;
+    const GemmScratch ws{l.gemm, l.gemm_bytes};
+    const int64_t kbp = padded_blocks(K);
+    if (M <= 128) {
+        SharedActGroups sg{};
+        sg.groups = G;
+        sg.tile_start[0] = 0;
+        for (int g = 0; g < G; ++g) {
+            sg.tile_start[g + 1] = sg.tile_start[g] + static_cast<int>(N[g] / 128);
+            sg.a_row[g] = static_cast<int>(g * seg);
+        }
+        return with_config(M, [&](auto bn, auto stages, auto sw) -> int {
+            if constexpr (decltype(sw)::value) {
+                GemmOperands op{Wq, Ws, l.Aq, l.As, n_total, M, K, y, n_total, 0};
+                op.q_map_rows = (G - 1) * seg + M;
+                return launch_gemm<decltype(bn)::value, decltype(stages)::value, true, SharedActGroups>(op, ws, st,
+                                                                                                        true, sg);
+            } else {
+                return MACAQ_EINVAL;  // not reached: up to 128 tokens always take a swap-AB configuration
+            }
+        });
+    }
+    int64_t n0 = 0;
+    for (int g = 0; g < G; ++g) {
+        const int64_t a0 = g * seg;
+        // only the first GEMM is a programmatic dependent (of the quantiser); the rest follow the
+        // GEMM before them in plain stream order, as they share its stream-K scratch
+        if (int r = run_mxfp4_gemm(l.Aq + a0 * (K / 2), l.As + (a0 / 128) * 128 * kbp, M, Wq + n0 * (K / 2),
+                                   Ws + (n0 / 128) * 128 * kbp, N[g], K, y + n0, 0, ws, st, g == 0, n_total))
+            return r;
+        n0 += N[g];
+    }
+    return MACAQ_OK;
 }
 
 // The group table of a grouped linear from the host token counts: tokens per expert, their rows in
@@ -1741,6 +1820,41 @@ extern "C" int macaq_w4a4_grouped_linear(const uint16_t* x, const int64_t* count
     }
     const GemmOperands op{Aq, As, Wq, Ws, P, E * N, K, y, N, 0};
     return launch_gemm<256, 4, false, GroupTable>(op, none, st, true, gt, &gs);
+}
+
+// Shape checks of the stacked-linears call; the total of the N[g] in *n_total.
+static int check_multi(int64_t M, int64_t K, int G, const int64_t* N, int64_t* n_total) {
+    if (int st = check_shape(M, K)) return st;
+    if (G < 1 || G > kMaxGroups) return MACAQ_ESHAPE;
+    if (static_cast<int64_t>(G) * ((M + 127) / 128 * 128) > kMaxDim) return MACAQ_ESHAPE;
+    int64_t t = 0;
+    for (int g = 0; g < G; ++g) {
+        if (N[g] < 128 || N[g] % 128 != 0 || N[g] > kMaxDim) return MACAQ_ESHAPE;
+        t += N[g];
+        if (t > kMaxDim) return MACAQ_ESHAPE;
+    }
+    *n_total = t;
+    return MACAQ_OK;
+}
+
+extern "C" size_t macaq_linear_multi_workspace_bytes(int64_t M, int G, int64_t K) {
+    if (check_shape(M, K) || G < 1 || G > kMaxGroups || static_cast<int64_t>(G) * ((M + 127) / 128 * 128) > kMaxDim)
+        return 0;
+    return multi_workspace_layout(nullptr, M, G, K).bytes;
+}
+
+extern "C" int macaq_w4a4_linear_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult,
+                                       const uint8_t* Wq, const uint8_t* Ws, const int64_t* N, uint16_t* y,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+    if (!x || !Wq || !Ws || !N || !y || !workspace) return MACAQ_EINVAL;
+    int64_t n_total = 0;
+    if (int st = check_multi(M, K, G, N, &n_total)) return st;
+    if (!aligned16(x) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y) || !aligned16(workspace) ||
+        (act_mult && !aligned16(act_mult)))
+        return MACAQ_EALIGN;
+    const MultiWorkspace l = multi_workspace_layout(workspace, M, G, K);
+    if (workspace_bytes < l.bytes) return MACAQ_EWORKSPACE;
+    return run_linear_multi(x, M, K, G, act_mult, Wq, Ws, N, n_total, y, l, static_cast<cudaStream_t>(stream));
 }
 
 #ifdef MACAQ_TEST_HOOKS

@@ -395,9 +395,13 @@ constexpr int64_t kAheadMinElems = int64_t(1) << 24;       // from here the tran
 
 // Thread = (run of `rpg` rows) x (block column kb) x (half hf), halves fastest, then columns;
 // the low half of a padded block column (kb >= K/32) writes the zero scale bytes of its rows.
+// blockIdx.y = g: the g-th of several linears on the same x, quantised with its own multipliers
+// (mult + g K) into rows g * seg_rows onwards of the codes and scales (one linear: g = 0).  With
+// seg_rows a multiple of 128 that segment's scale atoms are those of rows 0.. shifted by
+// seg_rows * padded_blocks(K) bytes, so both offsets are applied to the base pointers once.
 __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_kernel(
     const uint16_t* __restrict__ x, int64_t R, int64_t K, int64_t rpg, const float* __restrict__ mult,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int64_t seg_rows) {
     griddep_launch_dependents();
     const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
@@ -407,6 +411,9 @@ __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_ke
     const int64_t r0 = ((item >> 1) / kbp) * rpg;
     if (r0 >= R) return;  // both lanes of a pair leave together: same block column, same rows
     const int64_t n = r0 + rpg < R ? rpg : R - r0;
+    const int64_t o0 = static_cast<int64_t>(blockIdx.y) * seg_rows;  // this linear's first output row
+    codes += o0 * (K / 2);
+    scales += o0 * kbp;
     if (kb >= kb_real) {
         if (hf == 0)
             for (int64_t r = r0; r < r0 + n; ++r) scales[scale_offset(r, kb, kbp)] = 0;
@@ -415,7 +422,7 @@ __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_ke
     const unsigned pair_mask = 3u << (threadIdx.x & 30u);
     const int64_t k0 = kb * 32 + hf * 16;
     float2 m[8];
-    const float4* mp = reinterpret_cast<const float4*>(mult + k0);
+    const float4* mp = reinterpret_cast<const float4*>(mult + static_cast<int64_t>(blockIdx.y) * K + k0);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const float4 t = __ldg(mp + j);
@@ -428,18 +435,19 @@ __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_ke
         b[1] = __ldcs(p + 1);
     };
     auto out = [&](int64_t r) { return codes + r * (K / 2) + kb * 16 + hf * 8; };
+    auto sc = [&](int64_t r) { return scales + scale_offset(r, kb, kbp); };
     int64_t i = 0;
     for (; i + 1 < n; i += 2) {  // two rows at a time, both loaded before either is used
         uint4 b0[2], b1[2];
         load(r0 + i, b0);
         load(r0 + i + 1, b1);
-        half_block(b0, m, hf, pair_mask, out(r0 + i), scales + scale_offset(r0 + i, kb, kbp));
-        half_block(b1, m, hf, pair_mask, out(r0 + i + 1), scales + scale_offset(r0 + i + 1, kb, kbp));
+        half_block(b0, m, hf, pair_mask, out(r0 + i), sc(r0 + i));
+        half_block(b1, m, hf, pair_mask, out(r0 + i + 1), sc(r0 + i + 1));
     }
     if (i < n) {
         uint4 b0[2];
         load(r0 + i, b0);
-        half_block(b0, m, hf, pair_mask, out(r0 + i), scales + scale_offset(r0 + i, kb, kbp));
+        half_block(b0, m, hf, pair_mask, out(r0 + i), sc(r0 + i));
     }
 }
 
@@ -459,7 +467,7 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
         const int64_t rpg = half_rows_per_thread(M, K);
         const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
         mx_quant_half_kernel<<<static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads), kHalfThreads, 0,
-                               stream>>>(x, M, K, rpg, act_mult, Aq, As);
+                               stream>>>(x, M, K, rpg, act_mult, Aq, As, 0);
         return launch_status();
     }
     const int64_t rpg = quant_rows_per_thread(M, K);
@@ -509,6 +517,30 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
         mx_quant_grouped_kernel<QuantMode::kPlain><<<blocks, kQuantThreads, 0, stream>>>(x, K, nullptr, Aq, As, hg);
     }
     return launch_status();
+}
+
+// G linears on the same x (act_mult [G][K]): linear g's codes and scales are rows g * seg_rows to
+// g * seg_rows + M - 1 (seg_rows a multiple of 128, so each linear's scale atoms start a 128-row
+// block).  Small inputs: one half-block launch with a grid row per linear, its runs sized so all G
+// fit one resident wave; larger ones: the grouped quantiser with every group reading rows 0..M-1.
+int launch_act_transform_quant_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult,
+                                     int64_t seg_rows, uint8_t* Aq, uint8_t* As, cudaStream_t stream) {
+    if (M * K <= kHalfKernelMaxElems) {
+        const int64_t rpg = half_rows_per_thread(G * M, K);
+        const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
+        const dim3 grid(static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads), static_cast<unsigned>(G));
+        mx_quant_half_kernel<<<grid, kHalfThreads, 0, stream>>>(x, M, K, rpg, act_mult, Aq, As, seg_rows);
+        return launch_status();
+    }
+    GroupTable gt{};
+    gt.groups = G;
+    for (int g = 0; g < G; ++g) {
+        gt.rows[g] = static_cast<int>(M);
+        gt.x_row[g] = 0;
+        gt.a_row[g] = static_cast<int>(g * seg_rows);
+    }
+    gt.a_row[G] = static_cast<int>(G * seg_rows);
+    return launch_act_quant_grouped(x, K, act_mult, Aq, As, gt, stream);
 }
 
 // Rows per run of the grouped quantiser when only the total T of routed rows and the expert count

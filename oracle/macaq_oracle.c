@@ -6,10 +6,10 @@
  * shares no code, header, table or constant with the CUDA library.
  *
  * What it computes follows "MACaQ: Fast, Model Agnostic Calibrated Quantization for
- * Low-Precision Weights and Activations" (arXiv 2611.10649), Abstract: a per-channel
- * scale and a block-Hadamard transform are applied online to each layer's activations,
- * the corresponding inverse transforms are absorbed into the layer's weights, and both
- * sides are quantized to MXFP4 (W4A4), the weights by round-to-nearest.  The pages fix
+ * Low-Precision Weights and Activations" (arXiv 2611.10649), Abstract: at inference the
+ * activations of each layer are scaled channel by channel and rotated by a block
+ * Hadamard, the inverse of both is folded into that layer's weights, and both operands
+ * are MXFP4 (W4A4), the weights rounded to nearest.  The pages fix
  * neither the block size, the Hadamard normalisation, the scale direction, nor the MX
  * bit layout; the readings used here are:
  *
@@ -242,10 +242,10 @@ void oracle_mx_gemm(const uint8_t* Aq, const uint8_t* As, const int64_t* rows, i
 
 /* ------------------------------------------------------------------ Flip-Refinement
  *
- * "MACaQ ...", Abstract: to improve over round-to-nearest, Flip-Refinement is a Hessian-aware
- * coordinate-descent procedure that greedily moves individual FP4 codes to adjacent representable
- * values (the French news page adds: in place of GPTQ-style updates).  The pages give no more;
- * the readings used here:
+ * "MACaQ ...", Abstract: Flip-Refinement starts from the round-to-nearest codes and runs a greedy
+ * coordinate descent, weighted by the Hessian, in which a step shifts one FP4 code to a
+ * neighbouring grid value (the French news page sets it against GPTQ-style updates).  The pages
+ * give no more; the readings used here:
  *   - it refines one layer's folded weight codes W' = MXFP4(W diag(w) H_bd), starting from the
  *     round-to-nearest codes, with every E8M0 block scale kept (only codes move);
  *   - the objective of output row n is the layer's output error on the calibration batch,

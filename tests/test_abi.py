@@ -229,3 +229,36 @@ def test_validation_of_the_offline_and_grouped_device_calls():
     # layout conversions
     assert _call("macaq_scales_to_tiled", None, 4, 64, P(FAKE), None) == -1
     assert _call("macaq_scales_to_rowmajor", P(FAKE), 4, 48, P(FAKE), None) == -2
+
+
+def test_linear_multi_validation_and_sizes():
+    """The stacked-linears call refuses bad arguments before any CUDA call: null pointers, a layer
+    count or a layer width out of range, misalignment, a short workspace."""
+    import numpy as np
+    P = ctypes.c_void_p
+    lib = mq.load_library()
+    assert lib.macaq_linear_multi_workspace_bytes(16, 0, 512) == 0     # no layer
+    assert lib.macaq_linear_multi_workspace_bytes(16, 129, 512) == 0   # more than 128 layers
+    assert lib.macaq_linear_multi_workspace_bytes(16, 3, 48) == 0      # K % 32 != 0
+    # per layer 128 padded rows of codes (K/2 bytes each) and scales (8 * ceil(K/256) bytes each)
+    assert lib.macaq_linear_multi_workspace_bytes(16, 3, 512) >= 3 * 128 * (256 + 16)
+
+    def widths(*n):
+        a = np.array(n, dtype=np.int64)
+        return a, P(a.ctypes.data)
+
+    keep = []
+
+    def call(N=(256, 128, 128), G=None, x=FAKE, am=FAKE, y=FAKE, M=16, K=512, wsb=1 << 30):
+        a, ap = widths(*N)
+        keep.append(a)
+        return lib.macaq_w4a4_linear_multi(P(x), M, K, len(N) if G is None else G, P(am), P(FAKE), P(FAKE), ap,
+                                           P(y), P(FAKE), wsb, None)
+
+    assert lib.macaq_w4a4_linear_multi(P(FAKE), 16, 512, 3, P(FAKE), P(FAKE), P(FAKE), None, P(FAKE), P(FAKE),
+                                       1 << 30, None) == -1          # no widths
+    assert call(x=0) == -1 and call(y=0) == -1
+    assert call(G=0) == -2 and call(N=(256, 100)) == -2 and call(N=(256, 0)) == -2
+    assert call(M=0) == -2 and call(K=48) == -2
+    assert call(x=MIS) == -3 and call(am=MIS) == -3
+    assert call(wsb=1000) == -6

@@ -81,7 +81,8 @@ def test_summary_and_mx_diff_on_fake_results():
                          "llama3_8b_up_prefill": {"tflops": 4000.0, "linear_roofline": lr, **leg},
                          "qwen3_32b_up_decode_M1": {"gbs": 3600.0, "linear_roofline": lr, "vs_plain_mxfp4_pct": 2.0},
                          "qwen3_32b_stack": {"layers": 64, "M1": {"w4a4_ms": 6.5, "linear_roofline_frac": 0.4,
-                                                                  "vs_plain_mxfp4_pct": 3.0}},
+                                                                  "vs_plain_mxfp4_pct": 3.0,
+                                                                  "w4a4_one_linear_at_a_time_ms": 7.0}},
                          "qwen3_moe_grouped": {"experts": 128, "up_T16": {"ms": 0.015, "linear_roofline_frac": 0.5,
                                                                           "vs_plain_mxfp4_pct": 3.0}}},
            "parity": {"ok": True, "activations": {"exempt": 0}, "weights": {"exempt": 0}, "y_rel_fro_vs_oracle": 1e-6}}

@@ -3,8 +3,8 @@ the Hessian bit for bit, the refined codes bit for bit and the moves per row equ
 decision is taken in fp64 with the same operations in the same order on both sides (the reading
 in oracle/macaq_oracle.c), so the codes must agree exactly.
 
-"MACaQ ...", Abstract: Flip-Refinement greedily moves individual FP4 codes to adjacent
-representable values, Hessian-aware, to improve over round-to-nearest."""
+"MACaQ ...", Abstract: Flip-Refinement refines the round-to-nearest codes by a greedy,
+Hessian-weighted coordinate descent over single-code steps to neighbouring grid values."""
 import numpy as np
 import pytest
 import torch

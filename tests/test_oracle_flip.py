@@ -3,9 +3,8 @@ hand-derived worked cases, and properties that hold for any greedy descent of th
 checked against an objective written here from its definition (not the oracle's incremental
 arithmetic).
 
-"MACaQ ...", Abstract: Flip-Refinement is a Hessian-aware coordinate-descent procedure that
-greedily moves individual FP4 codes to adjacent representable values, improving on
-round-to-nearest.  Reading (oracle/macaq_oracle.c): per weight row the objective is
+"MACaQ ...", Abstract: Flip-Refinement refines the round-to-nearest codes by a greedy,
+Hessian-weighted coordinate descent over single-code steps to neighbouring grid values.  Reading (oracle/macaq_oracle.c): per weight row the objective is
 L = (q - v) Hs (q - v)^T with Hs = Xt^T Xt of the transformed calibration activations; block
 scales are kept; each step applies the single most-improving one-step move on the ordered E2M1
 value line; ties go to the smaller k, then the downward move."""
