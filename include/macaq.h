@@ -191,9 +191,10 @@ int macaq_mxfp4_gemm(const uint8_t* Aq, const uint8_t* As, int64_t M, const uint
  * macaq_w4a4_linear_multi -- G linear layers on the same activations x, e.g. the q, k and v
  * projections of an attention block or the gate and up projections of an MLP.  Each is its own
  * layer with its own per-channel scale and folded weights (the method is layer-local, Abstract),
- * so x is transformed and quantised once per layer, in ONE launch; then, for M <= 128, ONE
- * swap-AB GEMM runs over the layers' weights stacked by rows, each 128-row weight tile against
- * its own layer's activation tile (above 128 tokens, one GEMM per layer).
+ * so x is transformed and quantised once per layer, in ONE launch; then ONE GEMM runs over the
+ * layers' weights stacked by rows, each weight tile against its own layer's activations: up to
+ * 128 tokens swap-AB (128-row weight tiles), above on CTA pairs (256-row weight tiles) when every
+ * N[g] is a multiple of 256; otherwise one GEMM per layer.
  *   x         in   bf16 [M][K]
  *   act_mult  in   fp32 [G][K], layer g's multipliers from macaq_fold_weights at g*K; NULL: plain
  *                  MXFP4 of x, quantised once and shared (the "pure MXFP4" baseline)

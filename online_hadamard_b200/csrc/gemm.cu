@@ -799,11 +799,14 @@ __device__ __forceinline__ void pair_tile(const GemmParams& prm, int tile, int& 
     qt = local / rows;
 }
 
-template <int STAGES>
+// GT = SharedActGroups: stacked linears on one x (weights = B, stacked by rows; tile_start counts
+// 256-row weight tiles); each weight tile's activation panel is taken from its linear's segment.
+template <int STAGES, class GT = NoGroups>
 __global__ void __launch_bounds__(kPairThreads, 1)
     mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                           const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
-                          const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm) {
+                          const __grid_constant__ CUtensorMap tmap_y, const GemmParams prm,
+                          const __grid_constant__ GT gt) {
     using Cfg = PairCfg;
     constexpr int BN = 256;
     extern __shared__ uint8_t smem_raw[];
@@ -862,7 +865,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             while (!abort && it.next(prm, w)) {
                 int pt, qt;
                 pair_tile(prm, w.tile, pt, qt);
-                const int a_row = pt * 256 + static_cast<int>(rank) * 128;
+                int a_base = 0;  // first activation row of this tile's linear (a multiple of 128)
+                if constexpr (std::is_same<GT, SharedActGroups>::value)
+                    a_base = gt.a_row[group_of(gt.tile_start, gt.groups, qt)];
+                const int a_row = a_base + pt * 256 + static_cast<int>(rank) * 128;
                 const int b_row = qt * 256 + static_cast<int>(rank) * 128;
                 for (int kt = w.k0; kt < w.k1; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, &abort)) break;
@@ -873,7 +879,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     // scale atoms: 1 KB (two 512-byte atoms) per 128 rows per K step, as uint32 boxes
                     uint8_t* sf = sb + Cfg::kCodeBytes;
                     mbar_arrive_expect_tx(&sf_smem[stage], Cfg::kSFABytes + Cfg::kSFBBytes);
-                    tma_load_2d(sf, &tmap_sfa, kt * 256, 2 * pt + static_cast<int>(rank), &sf_smem[stage]);
+                    tma_load_2d(sf, &tmap_sfa, kt * 256, a_base / 128 + 2 * pt + static_cast<int>(rank),
+                                &sf_smem[stage]);
                     tma_load_2d(sf + 1024, &tmap_sfb, kt * 256, 2 * qt, &sf_smem[stage]);
                     tma_load_2d(sf + 2048, &tmap_sfb, kt * 256, 2 * qt + 1, &sf_smem[stage]);
                     if (++stage == STAGES) {
@@ -1195,6 +1202,7 @@ struct GemmOperands {
     int64_t ldy;
     int y_fp32;
     int64_t q_map_rows = 0;  // rows of Q's codes and scales if more than q_rows (stacked linears)
+    int64_t p_map_rows = 0;  // the same for P (pair kernel: the activations)
 };
 
 // Scratch of the stream-K schedule (nullptr: data-parallel schedule only).
@@ -1355,10 +1363,34 @@ static int pair_raster_group(int p_tiles, int pairs) {
     return g < p_tiles ? g : p_tiles;
 }
 
-static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int pairs, cudaStream_t stream, bool pdl) {
+// Shared-memory attributes of a pair-kernel instantiation other than the plain one (which
+// gemm_pairs_query sets), once per device.
+template <class GT>
+static bool pair_kernel_attributes() {
+    static int cache[64] = {0};
+    return cached_per_device(cache, [] {
+               auto kernel = mxf4_gemm_pair_kernel<kPairStages, GT>;
+               cudaFuncAttributes fa;
+               if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || !register_split_fits(fa)) {
+                   cudaGetLastError();
+                   return -1;
+               }
+               return (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pair_smem_bytes()) ==
+                           cudaSuccess &&
+                       cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100) == cudaSuccess)
+                          ? 1
+                          : -1;
+           }) == 1;
+}
+
+template <class GT = NoGroups>
+static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int pairs, cudaStream_t stream, bool pdl,
+                            const GT& groups = GT{}) {
+    if (!std::is_same<GT, NoGroups>::value && !pair_kernel_attributes<GT>()) return MACAQ_ECUDA;
+    const int64_t p_map_rows = op.p_map_rows > op.p_rows ? op.p_map_rows : op.p_rows;
     CUtensorMap ma, mb, msa, msb, my;
-    if (!make_codes_map(&ma, op.pq, op.p_rows, op.K, 128) || !make_codes_map(&mb, op.qq, op.q_rows, op.K, 128) ||
-        !make_sf_map(&msa, op.ps, op.p_rows, op.K) || !make_sf_map(&msb, op.qs, op.q_rows, op.K))
+    if (!make_codes_map(&ma, op.pq, p_map_rows, op.K, 128) || !make_codes_map(&mb, op.qq, op.q_rows, op.K, 128) ||
+        !make_sf_map(&msa, op.ps, p_map_rows, op.K) || !make_sf_map(&msb, op.qs, op.q_rows, op.K))
         return MACAQ_ECUDA;
     GemmParams prm{};
     prm.sf_p = op.ps;
@@ -1410,7 +1442,8 @@ static int launch_gemm_pair(const GemmOperands& op, const GemmScratch& ws, int p
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    if (cudaLaunchKernelEx(&cfg, mxf4_gemm_pair_kernel<kPairStages>, ma, mb, msa, msb, my, prm) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, mxf4_gemm_pair_kernel<kPairStages, GT>, ma, mb, msa, msb, my, prm, groups) !=
+        cudaSuccess)
         return MACAQ_ECUDA;
     return launch_status();
 }
@@ -1524,10 +1557,12 @@ static MultiWorkspace multi_workspace_layout(void* base, int64_t M, int G, int64
     return l;
 }
 
-// One quantiser launch for all G linears; then, up to 128 tokens, ONE swap-AB GEMM over the
-// stacked weights (each 128-row weight tile paired with its own linear's activation tile), so the
-// small k / v weights share the grid with the rest instead of each running on a few SMs; above
-// 128 tokens one GEMM per linear, each into its column block of y.
+// One quantiser launch for all G linears; then ONE GEMM over the stacked weights, each weight tile
+// paired with its own linear's activations, so the small k / v weights share the grid (and its
+// waves) with the rest instead of each running on a few SMs: up to 128 tokens swap-AB with
+// 128-row weight tiles, above on CTA pairs with 256-row weight tiles when every N[g] is a multiple
+// of 256 (a tile then never spans two linears).  Otherwise one GEMM per linear, each into its
+// column block of y.
 static int run_linear_multi(const uint16_t* x, int64_t M, int64_t K, int G, const float* act_mult, const uint8_t* Wq,
                             const uint8_t* Ws, const int64_t* N, int64_t n_total, uint16_t* y,
                             const MultiWorkspace& l, cudaStream_t st) {
@@ -1555,6 +1590,20 @@ static int run_linear_multi(const uint16_t* x, int64_t M, int64_t K, int G, cons
                 return MACAQ_EINVAL;  // not reached: up to 128 tokens always take a swap-AB configuration
             }
         });
+    }
+    bool whole_pair_tiles = true;
+    for (int g = 0; g < G; ++g) whole_pair_tiles = whole_pair_tiles && N[g] % 256 == 0;
+    if (use_pairs(M) && whole_pair_tiles) {
+        SharedActGroups sg{};
+        sg.groups = G;
+        sg.tile_start[0] = 0;
+        for (int g = 0; g < G; ++g) {
+            sg.tile_start[g + 1] = sg.tile_start[g] + static_cast<int>(N[g] / 256);
+            sg.a_row[g] = static_cast<int>(g * seg);
+        }
+        GemmOperands op{l.Aq, l.As, Wq, Ws, M, n_total, K, y, n_total, 0};
+        op.p_map_rows = (G - 1) * seg + M;
+        return launch_gemm_pair(op, ws, gemm_pairs(), st, true, sg);
     }
     int64_t n0 = 0;
     for (int g = 0; g < G; ++g) {

@@ -94,47 +94,60 @@ def _check(mq, layers, M, plain=False, col_sample=None):
 
 
 QKV_SMALL = _layers("qkv_small", 512, (512, 128, 128))
+QKV_PAIR = _layers("qkv_pair", 768, (512, 256, 256))
 
 
 @pytest.mark.parametrize("M", [1, 5, 16, 33, 64, 128, 129, 300])
 def test_stacked_qkv_small(mq, M):
-    """Every swap-AB tile width (M <= 128: one stacked GEMM, three activation segments) and the
-    per-layer GEMMs above 128 tokens (ragged M, y written with a row stride of sum N)."""
+    """Every swap-AB tile width (M <= 128: one stacked GEMM, three activation segments) and, above
+    128 tokens with a layer width that is not a multiple of 256, one GEMM per layer (ragged M, y
+    written with a row stride of sum N)."""
     _check(mq, QKV_SMALL, M)
+
+
+@pytest.mark.parametrize("M", [129, 300, 600])
+def test_stacked_pair_gemm(mq, M):
+    """Above 128 tokens with every width a multiple of 256: one CTA-pair GEMM over the stacked
+    weights, each 256-row weight tile against its layer's activation segment (ragged M: the
+    segments' padding rows and the next segment's rows reach only unstored output rows)."""
+    _check(mq, QKV_PAIR, M)
 
 
 def test_stacked_gate_up_ragged(mq):
     _check(mq, _layers("gateup_small", 1056, (384, 384)), 7)  # K = 33 blocks: a ragged 256-wide K tile
 
 
-@pytest.mark.parametrize("M", [16, 200])
-def test_stacked_plain_shares_one_quantisation(mq, M):
+@pytest.mark.parametrize("layers,M", [(QKV_SMALL, 16), (QKV_SMALL, 200), (QKV_PAIR, 300)])
+def test_stacked_plain_shares_one_quantisation(mq, layers, M):
     """act_mult = NULL: plain MXFP4 of x, quantised once, contracted with every layer's weights."""
-    _check(mq, QKV_SMALL, M, plain=True)
+    _check(mq, layers, M, plain=True)
 
 
-@pytest.mark.parametrize("M", [1, 16])
-def test_stacked_qwen_qkv_decode(mq, M):
-    """Qwen3-32B-shaped q, k and v projections (K = 5120; N = 8192, 1024, 1024) at decode: one
-    quantiser and one GEMM over 10240 stacked weight rows; sampled output columns."""
+@pytest.mark.parametrize("M", [1, 16, 512])
+def test_stacked_qwen_qkv(mq, M):
+    """Qwen3-32B-shaped q, k and v projections (K = 5120; N = 8192, 1024, 1024) at decode and at
+    512 tokens: one quantiser and one GEMM over 10240 stacked weight rows; sampled output columns."""
     layers = [wls.stack_layer(0, n, 1) for n in ("q", "k", "v")]
     _check(mq, layers, M, col_sample=512)
 
 
-def test_stacked_matches_single_layer_calls(mq):
-    """Above 128 tokens each layer runs the single layer's GEMM with the same schedule, so its
-    column block equals macaq_w4a4_linear's output bit for bit; at decode they agree within the
-    GEMM tolerance (the stacked launch splits the K steps over a different tile count)."""
-    for M in (16, 300):
-        x, y, Wq, Ws, am = _check(mq, QKV_SMALL, M)
-        n0, kb = 0, 8 * ((512 + 255) // 256)
-        for g, wl in enumerate(QKV_SMALL):
-            ys = mq.macaq_w4a4_linear(x.cuda(), am[g].contiguous(), Wq[n0:n0 + wl.N].contiguous(),
-                                      Ws[n0 * kb: (n0 + wl.N) * kb].contiguous(), wl.N)
-            torch.cuda.synchronize()
-            blk = y[:, n0:n0 + wl.N]
-            if M > 128:
-                assert torch.equal(blk, ys)
-            else:
-                assert gu.rel_fro(gu.to_np(blk.float()), gu.to_np(ys.float())) <= 1e-3
-            n0 += wl.N
+@pytest.mark.parametrize("layers,M", [(QKV_SMALL, 16), (QKV_SMALL, 300), (QKV_PAIR, 300)])
+def test_stacked_matches_single_layer_calls(mq, layers, M):
+    """Where each layer runs its own GEMM (above 128 tokens, a width not a multiple of 256) the
+    schedule is the single layer's, so its column block equals macaq_w4a4_linear's output bit for
+    bit; the stacked launches agree with it within the GEMM tolerance (they split the K steps over
+    a different tile count)."""
+    x, y, Wq, Ws, am = _check(mq, layers, M)
+    K = layers[0].K
+    n0, kb = 0, 8 * ((K + 255) // 256)
+    per_layer = M > 128 and any(wl.N % 256 for wl in layers)
+    for g, wl in enumerate(layers):
+        ys = mq.macaq_w4a4_linear(x.cuda(), am[g].contiguous(), Wq[n0:n0 + wl.N].contiguous(),
+                                  Ws[n0 * kb: (n0 + wl.N) * kb].contiguous(), wl.N)
+        torch.cuda.synchronize()
+        blk = y[:, n0:n0 + wl.N]
+        if per_layer:
+            assert torch.equal(blk, ys)
+        else:
+            assert gu.rel_fro(gu.to_np(blk.float()), gu.to_np(ys.float())) <= 1e-3
+        n0 += wl.N
