@@ -60,7 +60,7 @@ def _workspace_acts(ws, M, K, G, g):
     return gu.to_np(codes), gu.to_np(scales)
 
 
-def _check(mq, layers, M, plain=False, col_sample=None):
+def _check(mq, layers, M, plain=False, col_sample=None, row_sample=None):
     K = layers[0].K
     Ns = [wl.N for wl in layers]
     G = len(Ns)
@@ -72,6 +72,7 @@ def _check(mq, layers, M, plain=False, col_sample=None):
     xf = x.float().numpy()
     yg = gu.to_np(y.float())
     rng = np.random.default_rng(7000 + M)
+    rows = np.arange(M) if row_sample is None else np.sort(rng.choice(M, row_sample, replace=False))
     n0 = 0
     for g, (wl, (rWq, rWs, ra)) in enumerate(zip(layers, ref)):
         if plain:
@@ -84,8 +85,8 @@ def _check(mq, layers, M, plain=False, col_sample=None):
                           (lambda: xf.astype(np.float32)) if plain else (lambda ra=ra: oracle.transform_f32(xf, ra)),
                           label=f"config {MULTI_CONFIG} stacked-layers activations")
         cols = np.arange(wl.N) if col_sample is None else np.sort(rng.choice(wl.N, col_sample, replace=False))
-        want = oracle.mx_gemm(rAq, rAs, rWq[cols], rWs[cols])
-        got = yg[:, n0 + cols]
+        want = oracle.mx_gemm(rAq, rAs, rWq[cols], rWs[cols], rows=rows)
+        got = yg[rows][:, n0 + cols]
         err = gu.rel_fro(got, gu.bf16_round(want))
         print(f"layer {g} (N={wl.N}) M={M}{' plain' if plain else ''}: vs oracle {err:.2e}")
         assert err <= 1e-3
@@ -129,6 +130,15 @@ def test_stacked_qwen_qkv(mq, M):
     512 tokens: one quantiser and one GEMM over 10240 stacked weight rows; sampled output columns."""
     layers = [wls.stack_layer(0, n, 1) for n in ("q", "k", "v")]
     _check(mq, layers, M, col_sample=512)
+
+
+@pytest.mark.parametrize("M", [32, 4096])
+def test_stacked_qwen_gate_up(mq, M):
+    """Qwen3-32B-shaped gate and up projections (K = 5120, N = 25600 each): 51200 stacked weight rows,
+    swap-AB at 32 tokens, the CTA-pair GEMM with stream-K at 4096; every activation code and scale
+    compared, outputs on sampled rows and columns."""
+    layers = [wls.stack_layer(0, n, 1) for n in ("gate", "up")]
+    _check(mq, layers, M, col_sample=384, row_sample=None if M <= 64 else 48)
 
 
 @pytest.mark.parametrize("layers,M", [(QKV_SMALL, 16), (QKV_SMALL, 300), (QKV_PAIR, 300)])
