@@ -696,9 +696,37 @@ def summary(out):
     return sm
 
 
+def profile_stacked(name):
+    """Launch sequence for ncu of a stacked call of the 64-layer stack's first layer
+    ("qwen3_32b_stack_qkv_M<m>" or "qwen3_32b_stack_gateup_M<m>"): fold its layers into one stacked
+    buffer, then 3 x macaq_w4a4_linear_multi (one quantiser and one stacked GEMM each)."""
+    import online_hadamard_b200 as mq
+    base, _, m = name.partition("_M")
+    names = {"qwen3_32b_stack_qkv": ("q", "k", "v"), "qwen3_32b_stack_gateup": ("gate", "up")}[base]
+    M = int(m)
+    layers = [wls.stack_layer(0, n, M) for n in names]
+    K, Ns = layers[0].K, [wl.N for wl in layers]
+    folds = []
+    for wl in layers:
+        W = wls.make_w_device(wl, "cuda")
+        s = mq.macaq_calibrate_scale(wls.make_x_device(wl, wls.CALIB_TOKENS, "cuda", tensor_id=2), W)
+        folds.append(mq.macaq_fold_weights(W, s))
+        del W
+    Wq, Ws, am = torch.cat([f[0] for f in folds]), torch.cat([f[1] for f in folds]), torch.stack([f[2] for f in folds])
+    x = wls.make_x_device(layers[0], M, "cuda")
+    ws = torch.empty(mq.linear_multi_workspace_bytes(M, len(Ns), K), dtype=torch.uint8, device="cuda")
+    y = torch.empty(M, sum(Ns), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        mq.macaq_w4a4_linear_multi(x, am, Wq, Ws, Ns, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    print(f"profiled {base} M={M} K={K} N={'+'.join(map(str, Ns))}")
+
+
 def profile_kernels(name):
     """Launch sequence for ncu: fold once, then 3 x (transform+quant, plain quant, GEMM)."""
     import online_hadamard_b200 as mq
+    if name.startswith("qwen3_32b_stack_"):
+        return profile_stacked(name)
     base, _, m = name.partition("_M")
     wl = next(w for w in wls.ALL if w.name == base)
     if m:

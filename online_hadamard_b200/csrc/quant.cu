@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_kernel(
     const float* __restrict__ s, double c, float* __restrict__ act_mult_out, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales) {
     griddep_launch_dependents();
+    griddep_wait();  // x (and this workspace) may be written / still read by the preceding kernel
     const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
@@ -263,6 +264,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
     uint8_t* __restrict__ scales, const __grid_constant__ SRC src) {
     static_assert(MODE != QuantMode::kWeightFold, "activations only");
     griddep_launch_dependents();
+    griddep_wait();  // x (and this workspace) may be written / still read by the preceding kernel
     // A device-built table is copied to shared memory first: each thread's expert lookup is a binary
     // search, which would otherwise be a chain of dependent global loads.
     constexpr bool kDevTable = std::is_same<SRC, DeviceGroups>::value;
@@ -302,6 +304,27 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
         }
     }
     quant_rows<MODE, AHEAD>(x, K, gt.x_row[e] + t0, out0, n, kb, kbp, m, codes, scales);
+}
+
+// Activation quantisers are launched as programmatic dependents of whatever precedes them on the
+// stream (in a model, the previous layer's GEMM), so the launch is processed while that kernel's
+// last CTAs finish; each kernel's first act is griddepcontrol.wait, which returns once the
+// preceding grid has completed and its writes are visible, before x is read or the workspace
+// written.  After a copy or with nothing before it the attribute has no effect.  (Measured on
+// back-to-back decode linears: 0.3-0.7 us less per call.)
+template <class Kern, class... Args>
+static int launch_dependent(Kern kernel, dim3 grid, dim3 block, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return MACAQ_ECUDA;
+    return launch_status();
 }
 
 // Rows per thread: enough threads to fill the GPU, rows walked by each otherwise.
@@ -403,6 +426,7 @@ __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_ke
     const uint16_t* __restrict__ x, int64_t R, int64_t K, int64_t rpg, const float* __restrict__ mult,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int64_t seg_rows) {
     griddep_launch_dependents();
+    griddep_wait();  // x (and this workspace) may be written / still read by the preceding kernel
     const int64_t kb_real = K / 32;
     const int64_t kbp = padded_blocks(K);
     const int64_t item = static_cast<int64_t>(blockIdx.x) * kHalfThreads + threadIdx.x;
@@ -466,16 +490,14 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
     if (M * K <= kHalfKernelMaxElems) {
         const int64_t rpg = half_rows_per_thread(M, K);
         const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
-        mx_quant_half_kernel<<<static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads), kHalfThreads, 0,
-                               stream>>>(x, M, K, rpg, act_mult, Aq, As, 0);
-        return launch_status();
+        return launch_dependent(mx_quant_half_kernel, dim3(static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads)),
+                                dim3(kHalfThreads), stream, x, M, K, rpg, act_mult, Aq, As, int64_t(0));
     }
     const int64_t rpg = quant_rows_per_thread(M, K);
     const auto kernel = M * K >= kAheadMinElems ? mx_quant_kernel<QuantMode::kActTransform, true>
                                                 : mx_quant_kernel<QuantMode::kActTransform, false>;
-    kernel<<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(x, M, K, rpg, act_mult, nullptr, 0.0, nullptr, Aq,
-                                                                  As);
-    return launch_status();
+    return launch_dependent(kernel, dim3(quant_blocks(M, K, rpg)), dim3(kQuantThreads), stream, x, M, K, rpg, act_mult,
+                            static_cast<const float*>(nullptr), 0.0, static_cast<float*>(nullptr), Aq, As);
 }
 
 int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult, uint8_t* Aq, uint8_t* As,
@@ -512,11 +534,10 @@ int launch_act_quant_grouped(const uint16_t* x, int64_t K, const float* act_mult
     if (act_mult) {
         const auto kernel = tokens * K >= kAheadMinElems ? mx_quant_grouped_kernel<QuantMode::kActTransform, true>
                                                          : mx_quant_grouped_kernel<QuantMode::kActTransform, false>;
-        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, hg);
-    } else {
-        mx_quant_grouped_kernel<QuantMode::kPlain><<<blocks, kQuantThreads, 0, stream>>>(x, K, nullptr, Aq, As, hg);
+        return launch_dependent(kernel, dim3(blocks), dim3(kQuantThreads), stream, x, K, act_mult, Aq, As, hg);
     }
-    return launch_status();
+    return launch_dependent(mx_quant_grouped_kernel<QuantMode::kPlain>, dim3(blocks), dim3(kQuantThreads), stream, x,
+                            K, static_cast<const float*>(nullptr), Aq, As, hg);
 }
 
 // G linears on the same x (act_mult [G][K]): linear g's codes and scales are rows g * seg_rows to
@@ -529,8 +550,8 @@ int launch_act_transform_quant_multi(const uint16_t* x, int64_t M, int64_t K, in
         const int64_t rpg = half_rows_per_thread(G * M, K);
         const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
         const dim3 grid(static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads), static_cast<unsigned>(G));
-        mx_quant_half_kernel<<<grid, kHalfThreads, 0, stream>>>(x, M, K, rpg, act_mult, Aq, As, seg_rows);
-        return launch_status();
+        return launch_dependent(mx_quant_half_kernel, grid, dim3(kHalfThreads), stream, x, M, K, rpg, act_mult, Aq, As,
+                                seg_rows);
     }
     GroupTable gt{};
     gt.groups = G;
@@ -568,20 +589,18 @@ int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t
         const auto kernel = T * K >= kAheadMinElems
                                 ? mx_quant_grouped_kernel<QuantMode::kActTransform, true, DeviceGroups>
                                 : mx_quant_grouped_kernel<QuantMode::kActTransform, false, DeviceGroups>;
-        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, dg);
-    } else {
-        mx_quant_grouped_kernel<QuantMode::kPlain, false, DeviceGroups><<<blocks, kQuantThreads, 0, stream>>>(
-            x, K, nullptr, Aq, As, dg);
+        return launch_dependent(kernel, dim3(blocks), dim3(kQuantThreads), stream, x, K, act_mult, Aq, As, dg);
     }
-    return launch_status();
+    return launch_dependent(mx_quant_grouped_kernel<QuantMode::kPlain, false, DeviceGroups>, dim3(blocks),
+                            dim3(kQuantThreads), stream, x, K, static_cast<const float*>(nullptr), Aq, As, dg);
 }
 
 int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
                            cudaStream_t stream) {
     const int64_t rpg = quant_rows_per_thread(M, K);
-    mx_quant_kernel<QuantMode::kPlain><<<quant_blocks(M, K, rpg), kQuantThreads, 0, stream>>>(
-        x, M, K, rpg, nullptr, nullptr, 0.0, nullptr, Aq, As);
-    return launch_status();
+    return launch_dependent(mx_quant_kernel<QuantMode::kPlain>, dim3(quant_blocks(M, K, rpg)), dim3(kQuantThreads),
+                            stream, static_cast<const void*>(x), M, K, rpg, static_cast<const float*>(nullptr),
+                            static_cast<const float*>(nullptr), 0.0, static_cast<float*>(nullptr), Aq, As);
 }
 
 }  // namespace macaq
