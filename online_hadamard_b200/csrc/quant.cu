@@ -311,7 +311,11 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
 // last CTAs finish; each kernel's first act is griddepcontrol.wait, which returns once the
 // preceding grid has completed and its writes are visible, before x is read or the workspace
 // written.  After a copy or with nothing before it the attribute has no effect.  (Measured on
-// back-to-back decode linears: 0.3-0.7 us less per call.)
+// back-to-back decode linears: 0.3-0.7 us less per call.)  A consequence for the GEMM launched
+// after such a quantiser: it can start before the kernel ahead of the quantiser has finished, so
+// the GEMM touches no memory a preceding kernel may write (weights included) before its own
+// dependency wait, apart from the device-built expert table, whose quantiser is therefore launched
+// in plain stream order (launch_act_quant_grouped_device).
 template <class Kern, class... Args>
 static int launch_dependent(Kern kernel, dim3 grid, dim3 block, cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg = {};
@@ -580,6 +584,10 @@ int64_t device_groups_rpg(int64_t T, int E, int64_t K) {
 }
 int64_t device_groups_max_runs(int64_t T, int E, int64_t rpg) { return T / rpg + E; }
 
+// Launched in plain stream order, not as a programmatic dependent: the grouped GEMM that follows
+// reads the expert table (written by the table kernel just before this one) in all its warps before
+// its own dependency wait, which is safe only if this kernel -- and so the GEMM, launched after it
+// started -- began after the table kernel had completed.
 int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t K, const float* act_mult, uint8_t* Aq,
                                     uint8_t* As, const DeviceGroups& dg, cudaStream_t stream) {
     const int64_t rpg = device_groups_rpg(T, E, K);
@@ -589,10 +597,12 @@ int launch_act_quant_grouped_device(const uint16_t* x, int64_t T, int E, int64_t
         const auto kernel = T * K >= kAheadMinElems
                                 ? mx_quant_grouped_kernel<QuantMode::kActTransform, true, DeviceGroups>
                                 : mx_quant_grouped_kernel<QuantMode::kActTransform, false, DeviceGroups>;
-        return launch_dependent(kernel, dim3(blocks), dim3(kQuantThreads), stream, x, K, act_mult, Aq, As, dg);
+        kernel<<<blocks, kQuantThreads, 0, stream>>>(x, K, act_mult, Aq, As, dg);
+    } else {
+        mx_quant_grouped_kernel<QuantMode::kPlain, false, DeviceGroups><<<blocks, kQuantThreads, 0, stream>>>(
+            x, K, nullptr, Aq, As, dg);
     }
-    return launch_dependent(mx_quant_grouped_kernel<QuantMode::kPlain, false, DeviceGroups>, dim3(blocks),
-                            dim3(kQuantThreads), stream, x, K, static_cast<const float*>(nullptr), Aq, As, dg);
+    return launch_status();
 }
 
 int launch_act_quant_plain(const uint16_t* x, int64_t M, int64_t K, uint8_t* Aq, uint8_t* As,
