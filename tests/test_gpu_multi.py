@@ -114,6 +114,23 @@ def test_stacked_pair_gemm(mq, M):
     _check(mq, QKV_PAIR, M)
 
 
+def test_stacked_large_k_at_128_tokens(mq):
+    """M * K above the half-block quantiser's range at 128 tokens (K = 33024, 129 blocks: a ragged
+    last K tile): the grouped quantiser writes the segments, the swap-AB GEMM reads them."""
+    _check(mq, _layers("large_k", 33024, (256, 128)), 128, col_sample=96)
+
+
+def test_single_layer_stack_is_the_linear(mq):
+    """G = 1: the stacked call is the single layer's linear (same codes; y within the GEMM tolerance,
+    bit for bit where both take the same schedule)."""
+    layers = _layers("one", 512, (384,))
+    for M in (3, 200):
+        x, y, Wq, Ws, am = _check(mq, layers, M)
+        ys = mq.macaq_w4a4_linear(x.cuda(), am[0].contiguous(), Wq, Ws, 384)
+        torch.cuda.synchronize()
+        assert gu.rel_fro(gu.to_np(y.float()), gu.to_np(ys.float())) <= 1e-3
+
+
 def test_stacked_gate_up_ragged(mq):
     _check(mq, _layers("gateup_small", 1056, (384, 384)), 7)  # K = 33 blocks: a ragged 256-wide K tile
 
