@@ -155,6 +155,10 @@ def test_binding_refuses_host_tensors_and_short_buffers():
     with pytest.raises(ValueError, match="CUDA tensor"):
         mq.macaq_w4a4_linear(x, torch.ones(256), torch.zeros(128, 128, dtype=torch.uint8),
                              torch.zeros(mq.scale_bytes(128, 256), dtype=torch.uint8), 128)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mq.macaq_w4a4_linear_multi(x, torch.ones(2, 256), torch.zeros(384, 128, dtype=torch.uint8),
+                                   torch.zeros(mq.scale_bytes(256, 256) + mq.scale_bytes(128, 256), dtype=torch.uint8),
+                                   (256, 128))
     with pytest.raises(ValueError, match="needs at least"):
         mq._need_numel(torch.zeros(mq.scale_bytes(128, 256) - 1, dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
     mq._need_numel(torch.zeros(mq.scale_bytes(128, 256), dtype=torch.uint8), "Ws", mq.scale_bytes(128, 256))
