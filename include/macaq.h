@@ -6,7 +6,8 @@
  * and Activations" (arXiv 2611.10649), Abstract: no linear layer depends on another; at
  * inference the activations of a layer are scaled channel by channel and rotated by a
  * block Hadamard, and the inverse of both is folded into the same layer's weights; both
- * operands are MXFP4 (W4A4), the weights rounded to nearest.  The pages leave the details open; this library fixes them as follows.
+ * operands are MXFP4 (W4A4), the weights rounded to nearest.  The pages leave the details
+ * open; this library fixes them as follows.
  *
  *   Notation.  x is bf16 [M][K] row-major, W is fp32 [N][K] row-major (y = x W^T, the
  *   nn.Linear layout), s is fp32 [K] with s_k > 0 finite.  c = 1/sqrt(32).

@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_kernel(
         const float4* mp = reinterpret_cast<const float4*>(mult + k0);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 t = __ldg(mp + j);
+            const float4 t = __ldcg(mp + j);  // through L2: launched before the kernel ahead ends
             m[2 * j] = make_float2(t.x, t.y);
             m[2 * j + 1] = make_float2(t.z, t.w);
         }
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kQuantThreads, 4) mx_quant_grouped_kernel(
         const float4* mp = reinterpret_cast<const float4*>(act_mult + static_cast<int64_t>(e) * K + kb * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 t = __ldg(mp + j);
+            const float4 t = __ldcg(mp + j);  // through L2: launched before the kernel ahead ends
             m[2 * j] = make_float2(t.x, t.y);
             m[2 * j + 1] = make_float2(t.z, t.w);
         }
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kHalfThreads, kHalfMinBlocks) mx_quant_half_ke
     const float4* mp = reinterpret_cast<const float4*>(mult + static_cast<int64_t>(blockIdx.y) * K + k0);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float4 t = __ldg(mp + j);
+        const float4 t = __ldcg(mp + j);  // through L2: launched before the kernel ahead ends
         m[2 * j] = make_float2(t.x, t.y);
         m[2 * j + 1] = make_float2(t.z, t.w);
     }
@@ -494,8 +494,9 @@ int launch_act_transform_quant(const uint16_t* x, int64_t M, int64_t K, const fl
     if (M * K <= kHalfKernelMaxElems) {
         const int64_t rpg = half_rows_per_thread(M, K);
         const int64_t items = 2 * padded_blocks(K) * ((M + rpg - 1) / rpg);
-        return launch_dependent(mx_quant_half_kernel, dim3(static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads)),
-                                dim3(kHalfThreads), stream, x, M, K, rpg, act_mult, Aq, As, int64_t(0));
+        const dim3 grid(static_cast<unsigned>((items + kHalfThreads - 1) / kHalfThreads));
+        return launch_dependent(mx_quant_half_kernel, grid, dim3(kHalfThreads), stream, x, M, K, rpg, act_mult, Aq, As,
+                                int64_t(0));
     }
     const int64_t rpg = quant_rows_per_thread(M, K);
     const auto kernel = M * K >= kAheadMinElems ? mx_quant_kernel<QuantMode::kActTransform, true>

@@ -38,7 +38,7 @@ def _rank_main(rank, world, port, out):
 
 def test_replicas_max_over_ranks_gloo():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
         res = dict(out)
